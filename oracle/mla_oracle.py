@@ -1,0 +1,260 @@
+"""fp64 CPU oracle for MLA decoding over a paged latent KV cache.
+
+TEST INFRASTRUCTURE. Only ``tests/``, ``__graft_entry__.smoke()`` and
+``bench.py``'s cpu_baseline / reference legs may import or run anything in this
+directory. The CUDA path never calls it and shares no code with it.
+
+What it computes (plain definition, no tiling, no online softmax). For request
+b, query token i in [0, s_q) and head h:
+  key set T  dense : { t : 0 <= t < seqlen_b }, and with the causal mask also
+                     t <= seqlen_b - s_q + i (the s_q queries are the request's
+                     last tokens);
+             sparse: the multiset { indices[b, i, k] : entry != -1 }.
+  row(t)   = cache[block_table[b, t // 64], t % 64, :]   (576 values)
+  s_t      = scale * <q[b, i, h, :], row(t)>             (K = all 576 dims)
+  m        = max_t s_t,   l = sum_t exp(s_t - m)
+  out      = sum_t exp(s_t - m) * row(t)[:512] / l        (V = first 512 dims)
+  lse      = m + ln(l)                                    (natural log)
+  empty T  : out = 0, lse = -inf   (the pages say nothing; chosen reading)
+
+Passages followed:
+  * FlashMLA-ETAP (gist.science summary), "핵심 메커니즘" (core mechanism):
+    S = Q K^T, P = softmax(S), O = P V.
+  * "[flashinfer] FlashInfer, NVFP4를 활용한 DeepSeek-V4 디코딩 성능 최적화",
+    section 2 (README of nvfp4_mla_decode): one latent row per token is both K
+    and V, 64-token pages, causal mask inside the q_len block against the
+    request's last tokens, natural-log FP32 LSE; tensor table (block_tables
+    [batch, max_pages], seq_lens [batch], out [.., 512] bf16, lse fp32).
+  * "Qu'est-ce que FlashMLA ?" (topnet.top), "Exécuter le décodage MLA": the
+    decode call takes q, the paged cache, block_table, cache_seqlens, dv and
+    causal.
+  * deepseek-ai/FlashMLA (agentlenshq), "기술적 세부 사항": indices entries of
+    -1 are ignored; FP8 cache = quantised values plus per-token scale factors.
+  * DeepSeek MLA geometry (FlashMLA-ETAP summary, limitations paragraph): 576
+    head dimension; the value part is the first 512 dims (dv = 512).
+
+Readings where the pages are silent (listed in the design doc as well):
+  * sparse indices are logical token positions of request b, resolved through
+    the block table; valid range [0, seqlen_b); any other value except -1 is
+    ignored and reported as out of range; duplicates count twice.
+  * FP8 record = [512 e4m3 | 4 fp32 scales | 64 bf16 RoPE]; the dequantised
+    value is bf16_RNE(fp32(e4m3) * scale) with the fp32 product rounded to
+    nearest; the oracle then uses those values exactly in fp64.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+PAGE = 64
+D_QK = 576
+D_V = 512
+FP8_TILE = 128
+FP8_RECORD_BYTES = 656
+
+
+# --------------------------------------------------------------------------
+# exact storage-format conversions
+# --------------------------------------------------------------------------
+def bf16_bits_to_f64(bits) -> np.ndarray:
+    """bf16 bit patterns (uint16) -> fp64. bf16 is the top half of an fp32."""
+    b = np.asarray(bits).astype(np.uint32) << np.uint32(16)
+    return b.view(np.float32).astype(np.float64)
+
+
+def torch_bf16_to_f64(t) -> np.ndarray:
+    """A torch bfloat16 tensor -> fp64 numpy array, via its bit patterns."""
+    import torch
+    assert t.dtype == torch.bfloat16
+    return bf16_bits_to_f64(t.contiguous().view(torch.int16).numpy().view(np.uint16))
+
+
+def f32_round_to_bf16(x) -> np.ndarray:
+    """fp32 -> nearest bf16 value (ties to even), returned as fp32.
+
+    Round-to-nearest-even on the 16 dropped mantissa bits; NaN stays NaN.
+    """
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    u = x.view(np.uint32).astype(np.uint64)
+    lsb = (u >> np.uint64(16)) & np.uint64(1)
+    r = ((u + np.uint64(0x7FFF) + lsb) & np.uint64(0xFFFF0000)).astype(np.uint32)
+    out = r.view(np.float32).copy()
+    nan = np.isnan(x)
+    out[nan] = np.nan
+    return out
+
+
+def e4m3_to_f64(codes) -> np.ndarray:
+    """OCP FP8 E4M3 ("fn": no infinities) code -> value.
+
+    sign bit 7, exponent bits 6..3 (bias 7), mantissa bits 2..0.
+    exponent 0: subnormal, value = m/8 * 2^-6; exponent 15 with mantissa 7:
+    NaN; otherwise (1 + m/8) * 2^(e-7). Largest finite magnitude 448.
+    """
+    c = np.asarray(codes).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = c & 0x7
+    val = np.where(e == 0, (m / 8.0) * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    val = sign * val
+    return np.where((e == 15) & (m == 7), np.nan, val)
+
+
+def dequant_fp8_records(records) -> np.ndarray:
+    """uint8 [P, 64, 656] token records -> fp64 [P, 64, 576] dequantised rows.
+
+    latent d (< 512): bf16_RNE(fp32(e4m3(code_d)) * scale[d // 128]) with the
+    fp32 product rounded to nearest; RoPE dims 512..575: the stored bf16.
+    """
+    rec = np.ascontiguousarray(np.asarray(records, dtype=np.uint8))
+    P = rec.shape[0]
+    codes = rec[..., :D_V]
+    scales = rec[..., D_V:D_V + 16].copy().view(np.float32)            # [P,64,4]
+    rope_bits = rec[..., D_V + 16:].copy().view(np.uint16)               # [P,64,64]
+    val = e4m3_to_f64(codes).astype(np.float32)                          # exact
+    sc = np.repeat(scales, FP8_TILE, axis=-1)                            # [P,64,512]
+    prod = (val * sc).astype(np.float32)                                 # fp32 RN product
+    lat = f32_round_to_bf16(prod).astype(np.float64)
+    out = np.empty((P, PAGE, D_QK), dtype=np.float64)
+    out[..., :D_V] = lat
+    out[..., D_V:] = bf16_bits_to_f64(rope_bits)
+    return out
+
+
+# --------------------------------------------------------------------------
+# the attention definition
+# --------------------------------------------------------------------------
+def attend(q_rows, keys, scale, d_v=D_V):
+    """softmax(scale * q_rows @ keys^T) @ keys[:, :d_v] and its natural-log LSE.
+
+    q_rows [R, d_qk], keys [T, d_qk] (T may be 0). Returns (out [R, d_v],
+    lse [R]). Empty key set: out 0, lse -inf.
+    """
+    q_rows = np.asarray(q_rows, dtype=np.float64)
+    keys = np.asarray(keys, dtype=np.float64)
+    R = q_rows.shape[0]
+    if keys.shape[0] == 0:
+        return np.zeros((R, d_v)), np.full(R, -np.inf)
+    s = scale * (q_rows @ keys.T)                        # [R, T]
+    m = s.max(axis=1, keepdims=True)
+    e = np.exp(s - m)
+    l = e.sum(axis=1, keepdims=True)
+    out = (e @ keys[:, :d_v]) / l
+    lse = m[:, 0] + np.log(l[:, 0])
+    return out, lse
+
+
+def gather_rows(cache_f64, block_table_row, positions):
+    """Rows of logical token positions of one request, through its block table.
+
+    cache_f64 [P, 64, d_qk]; block_table_row [max_pages]; positions int array.
+    """
+    positions = np.asarray(positions, dtype=np.int64)
+    pages = np.asarray(block_table_row, dtype=np.int64)[positions // PAGE]
+    return cache_f64[pages, positions % PAGE]
+
+
+def cache_to_f64(kcache) -> np.ndarray:
+    """Decode the cache storage (torch bf16 [P,64,1,576] or uint8 fp8 records)."""
+    import torch
+    if isinstance(kcache, torch.Tensor) and kcache.dtype == torch.bfloat16:
+        c = torch_bf16_to_f64(kcache)
+        return c.reshape(c.shape[0], PAGE, -1)
+    arr = kcache.numpy() if hasattr(kcache, "numpy") else np.asarray(kcache)
+    if arr.dtype == np.uint8:
+        return dequant_fp8_records(arr.reshape(arr.shape[0], PAGE, FP8_RECORD_BYTES))
+    arr = np.asarray(arr, dtype=np.float64)
+    return arr.reshape(arr.shape[0], PAGE, -1)
+
+
+def decode_dense(q, cache_f64, block_table, cache_seqlens, scale, causal,
+                 d_v=D_V, requests=None):
+    """Dense paged MLA decode. q [B, s_q, h_q, d_qk] (fp64 values).
+
+    Returns out [B, s_q, h_q, d_v] and lse [B, s_q, h_q] (requests not in
+    ``requests`` are left NaN when a subset is asked for).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    B, s_q, h_q, _ = q.shape
+    bt = np.asarray(block_table)
+    lens = np.asarray(cache_seqlens, dtype=np.int64)
+    out = np.full((B, s_q, h_q, d_v), np.nan)
+    lse = np.full((B, s_q, h_q), np.nan)
+    for b in (range(B) if requests is None else requests):
+        L = int(lens[b])
+        keys_all = gather_rows(cache_f64, bt[b], np.arange(L))
+        for i in range(s_q):
+            n = L
+            if causal:
+                n = max(0, min(L, L - s_q + i + 1))
+            o, l_ = attend(q[b, i], keys_all[:n], scale, d_v)
+            out[b, i], lse[b, i] = o, l_
+    return out, lse
+
+
+def sparse_key_positions(index_row, seqlen):
+    """Kept positions of one indices row, and the slots that were ignored.
+
+    -1 is ignored; any other value outside [0, seqlen) is ignored and counted
+    as out of range. Returns (positions, ignored_slots, out_of_range_slots).
+    """
+    r = np.asarray(index_row, dtype=np.int64)
+    valid = (r >= 0) & (r < seqlen)
+    oob = ~valid & (r != -1)
+    return r[valid], np.nonzero(~valid)[0], np.nonzero(oob)[0]
+
+
+def decode_sparse(q, cache_f64, block_table, cache_seqlens, indices, scale,
+                  d_v=D_V, requests=None):
+    """Token-sparse paged MLA decode; key set per (b, i) from indices[b, i]."""
+    q = np.asarray(q, dtype=np.float64)
+    B, s_q, h_q, _ = q.shape
+    bt = np.asarray(block_table)
+    lens = np.asarray(cache_seqlens, dtype=np.int64)
+    idx = np.asarray(indices)
+    out = np.full((B, s_q, h_q, d_v), np.nan)
+    lse = np.full((B, s_q, h_q), np.nan)
+    for b in (range(B) if requests is None else requests):
+        for i in range(s_q):
+            pos, _, _ = sparse_key_positions(idx[b, i], int(lens[b]))
+            keys = gather_rows(cache_f64, bt[b], pos)
+            o, l_ = attend(q[b, i], keys, scale, d_v)
+            out[b, i], lse[b, i] = o, l_
+    return out, lse
+
+
+def combine(o_parts, lse_parts):
+    """Merge attention results of disjoint key subsets (split-KV reduction).
+
+    o_parts [n, R, d] (each normalised over its own subset), lse_parts [n, R].
+    L = ln sum_s exp(lse_s); out = sum_s exp(lse_s - L) o_s. All parts empty:
+    out 0, lse -inf.
+    (FlashInfer PR #5443 analysis, section 3: a split-KV combine kernel merges
+    the partial results of CTAs that split one request's KV.)
+    """
+    o_parts = np.asarray(o_parts, dtype=np.float64)
+    lse_parts = np.asarray(lse_parts, dtype=np.float64)
+    mx = lse_parts.max(axis=0)
+    finite = np.isfinite(mx)
+    mxs = np.where(finite, mx, 0.0)
+    w = np.exp(lse_parts - mxs)                     # exp(-inf) = 0 for empty parts
+    tot = w.sum(axis=0)
+    L = np.where(finite, mxs + np.log(np.where(finite, tot, 1.0)), -np.inf)
+    wn = np.where(finite, w / np.where(finite, tot, 1.0), 0.0)
+    out = np.einsum("nr,nrd->rd", wn, o_parts)
+    return out, L
+
+
+def inputs_to_f64(inp):
+    """(q fp64, cache fp64) from a workloads.DecodeInputs."""
+    return torch_bf16_to_f64(inp.q), cache_to_f64(inp.kcache)
+
+
+def reference_decode(inp, requests=None):
+    """Run the oracle on a workloads.DecodeInputs; returns (out, lse) fp64."""
+    w = inp.workload
+    q, cache = inputs_to_f64(inp)
+    if w.topk:
+        return decode_sparse(q, cache, inp.block_table.numpy(), inp.cache_seqlens.numpy(),
+                             inp.indices.numpy(), w.scale, requests=requests)
+    return decode_dense(q, cache, inp.block_table.numpy(), inp.cache_seqlens.numpy(),
+                        w.scale, w.causal, requests=requests)

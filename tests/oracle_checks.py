@@ -1,0 +1,326 @@
+"""Independent pins for the fp64 oracle.
+
+Every check takes the oracle function(s) it exercises as arguments, so the
+same check can be run against the real oracle (must pass) and against planted
+mistakes (must fail; see test_oracle_mutants.py). None of the checks re-uses
+the oracle's own formulas: they use 50-digit mpmath brute force, closed forms,
+scipy's logsumexp, invariances, and torch's own fp8/bf16 conversions.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import mpmath
+import numpy as np
+import torch
+from scipy.special import logsumexp
+
+mpmath.mp.dps = 50
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+PAGE = 64
+
+
+# ---------------------------------------------------------------- helpers
+def _mp_attend(q_rows, keys, scale, d_v):
+    """Pure-Python 50-digit softmax attention (no numpy arithmetic)."""
+    R = len(q_rows)
+    outs, lses = [], []
+    for r in range(R):
+        s = [mpmath.mpf(scale) * mpmath.fsum(mpmath.mpf(float(a)) * mpmath.mpf(float(b))
+                                             for a, b in zip(q_rows[r], k)) for k in keys]
+        if not s:
+            outs.append([0.0] * d_v)
+            lses.append(-math.inf)
+            continue
+        m = max(s)
+        e = [mpmath.exp(x - m) for x in s]
+        l = mpmath.fsum(e)
+        o = [mpmath.fsum(e[t] * mpmath.mpf(float(keys[t][d])) for t in range(len(keys))) / l
+             for d in range(d_v)]
+        outs.append([float(v) for v in o])
+        lses.append(float(m + mpmath.log(l)))
+    return np.array(outs), np.array(lses)
+
+
+def _random_paged(rng, lens, d_qk, extra_pages=0):
+    """Small paged cache with a random physical page order (fp64 values)."""
+    npg = [(L + PAGE - 1) // PAGE for L in lens]
+    P = sum(npg) + extra_pages
+    perm = rng.permutation(P)
+    bt = np.full((len(lens), max(1, max(npg))), -1, dtype=np.int64)
+    off = 0
+    for b, n in enumerate(npg):
+        bt[b, :n] = perm[off:off + n]
+        off += n
+    cache = rng.standard_normal((P, PAGE, d_qk))
+    return cache, bt
+
+
+def _close(a, b, tol):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    assert a.shape == b.shape, (a.shape, b.shape)
+    both_inf = np.isinf(a) & np.isinf(b) & (np.sign(a) == np.sign(b))
+    err = np.where(both_inf, 0.0, np.abs(a - b) / (1.0 + np.abs(b)))
+    assert np.all(np.isfinite(err)) and err.max(initial=0.0) <= tol, f"max rel err {err.max()}"
+
+
+# ---------------------------------------------------------------- checks
+def check_brute_force_attend(attend, seeds=range(6)):
+    """attend() vs 50-digit brute force on tiny shapes (d_qk<=8, <=5 keys)."""
+    for seed in seeds:
+        rng = np.random.default_rng(seed)
+        d_qk, d_v = int(rng.integers(2, 9)), 0
+        d_v = int(rng.integers(1, d_qk + 1))
+        T = int(rng.integers(1, 6))
+        R = int(rng.integers(1, 4))
+        q = rng.standard_normal((R, d_qk)) * 2
+        k = rng.standard_normal((T, d_qk)) * 2
+        scale = float(rng.uniform(0.1, 1.5))
+        o, l = attend(q, k, scale, d_v)
+        eo, el = _mp_attend(q.tolist(), k.tolist(), scale, d_v)
+        _close(o, eo, 1e-13)
+        _close(l, el, 1e-13)
+
+
+def check_brute_force_paged(decode_dense, causal, seeds=range(3)):
+    """decode_dense() vs brute force that walks token by token through pages."""
+    for seed in seeds:
+        rng = np.random.default_rng(100 + seed)
+        d_qk, d_v = 6, 4
+        s_q = 2 if causal else 1
+        lens = [int(x) for x in rng.integers(1, 140, size=2)]
+        cache, bt = _random_paged(rng, lens, d_qk, extra_pages=1)
+        q = rng.standard_normal((2, s_q, 2, d_qk))
+        scale = 0.7
+        out, lse = decode_dense(q, cache, bt, np.array(lens), scale, causal, d_v=d_v)
+        for b, L in enumerate(lens):
+            for i in range(s_q):
+                last = L - s_q + i if causal else L - 1
+                keys = []
+                for t in range(0, max(0, last + 1)):
+                    page = bt[b][t // PAGE]
+                    keys.append(list(cache[page][t % PAGE]))
+                eo, el = _mp_attend(q[b, i].tolist(), keys, scale, d_v)
+                _close(out[b, i], eo, 1e-13)
+                _close(lse[b, i], el, 1e-13)
+
+
+def check_single_token(decode_dense, d_v=512):
+    """seqlen 1: out is that token's V row exactly; lse = scale * q.k."""
+    rng = np.random.default_rng(7)
+    d_qk = 576
+    cache, bt = _random_paged(rng, [1], d_qk, extra_pages=2)
+    q = rng.standard_normal((1, 1, 3, d_qk))
+    out, lse = decode_dense(q, cache, bt, np.array([1]), 1 / 24, False, d_v=d_v)
+    row = cache[bt[0][0], 0]
+    for h in range(3):
+        assert np.array_equal(out[0, 0, h], row[:d_v])
+        _close(lse[0, 0, h], (1 / 24) * float(np.dot(q[0, 0, h], row)), 1e-14)
+
+
+def check_constant_scores(decode_dense, d_v=512):
+    """Equal scores for every key: out = mean of V rows, lse = s + ln n.
+
+    q is zero on the first 512 dims, and every token shares the same RoPE part
+    (dims 512..575) while its latent part differs, so all scores are equal
+    but the V rows are not.
+    """
+    rng = np.random.default_rng(8)
+    d_qk, n = 576, 131
+    cache, bt = _random_paged(rng, [n], d_qk)
+    rope = rng.standard_normal(d_qk - 512)
+    cache[..., 512:] = rope
+    q = np.zeros((1, 1, 2, d_qk))
+    q[..., 512:] = rng.standard_normal((1, 1, 2, d_qk - 512))
+    out, lse = decode_dense(q, cache, bt, np.array([n]), 0.5, False, d_v=d_v)
+    rows = np.stack([cache[bt[0][t // PAGE], t % PAGE] for t in range(n)])
+    for h in range(2):
+        _close(out[0, 0, h], rows[:, :d_v].mean(axis=0), 1e-13)
+        s = 0.5 * float(np.dot(q[0, 0, h, 512:], rope))
+        _close(lse[0, 0, h], s + math.log(n), 1e-13)
+
+
+def check_lse_logsumexp(decode_dense):
+    """lse equals scipy's logsumexp of the explicit score vector."""
+    rng = np.random.default_rng(9)
+    d_qk = 576
+    lens = [200, 64, 1]
+    cache, bt = _random_paged(rng, lens, d_qk)
+    q = rng.standard_normal((3, 1, 4, d_qk))
+    _, lse = decode_dense(q, cache, bt, np.array(lens), 1 / 24, False)
+    for b, L in enumerate(lens):
+        for h in range(4):
+            sc = [(1 / 24) * math.fsum(q[b, 0, h] * cache[bt[b][t // PAGE], t % PAGE])
+                  for t in range(L)]
+            _close(lse[b, 0, h], logsumexp(sc), 1e-13)
+
+
+def check_page_permutation(decode_dense):
+    """Moving physical pages (and the block table with them) changes no bit."""
+    rng = np.random.default_rng(10)
+    d_qk = 576
+    lens = [70, 129, 5]
+    cache, bt = _random_paged(rng, lens, d_qk, extra_pages=3)
+    q = rng.standard_normal((3, 1, 2, d_qk))
+    o1, l1 = decode_dense(q, cache, bt, np.array(lens), 1 / 24, False)
+    P = cache.shape[0]
+    perm = rng.permutation(P)                 # new location of old page p = perm[p]
+    cache2 = np.empty_like(cache)
+    cache2[perm] = cache
+    bt2 = np.where(bt >= 0, perm[np.maximum(bt, 0)], -1)
+    o2, l2 = decode_dense(q, cache2, bt2, np.array(lens), 1 / 24, False)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+
+
+def check_causal_row0(decode_dense):
+    """s_q=2 causal: query 0 equals a non-causal run over seqlen-1 tokens,
+    query 1 equals a non-causal run over all seqlen tokens."""
+    rng = np.random.default_rng(11)
+    d_qk = 576
+    lens = [130, 65, 2]
+    cache, bt = _random_paged(rng, lens, d_qk)
+    q = rng.standard_normal((3, 2, 3, d_qk))
+    oc, lc = decode_dense(q, cache, bt, np.array(lens), 1 / 24, True)
+    o0, l0 = decode_dense(q[:, :1], cache, bt, np.array(lens) - 1, 1 / 24, False)
+    o1, l1 = decode_dense(q[:, 1:], cache, bt, np.array(lens), 1 / 24, False)
+    assert np.array_equal(oc[:, 0], o0[:, 0]) and np.array_equal(lc[:, 0], l0[:, 0])
+    assert np.array_equal(oc[:, 1], o1[:, 0]) and np.array_equal(lc[:, 1], l1[:, 0])
+
+
+def check_sparse(decode_sparse, decode_dense):
+    """-1 slots contribute nothing; all positions in order equals dense;
+    a shuffled index list gives the same result within fp64 rounding."""
+    rng = np.random.default_rng(12)
+    d_qk = 576
+    lens = [300, 129]
+    cache, bt = _random_paged(rng, lens, d_qk)
+    q = rng.standard_normal((2, 1, 3, d_qk))
+    # (a) -1 slots vs the compacted list (same order of kept entries)
+    topk = 128
+    idx = np.stack([rng.choice(L, size=topk, replace=False) for L in lens])[:, None, :]
+    holes = idx.copy()
+    holes[0, 0, rng.choice(topk, 17, replace=False)] = -1
+    holes[1, 0, :5] = -1
+    o_h, l_h = decode_sparse(q, cache, bt, np.array(lens), holes, 1 / 24)
+    for b in range(2):
+        kept = holes[b, 0][holes[b, 0] != -1]
+        o_c, l_c = decode_sparse(q[b:b + 1], cache, bt[b:b + 1], np.array(lens[b:b + 1]),
+                                 kept[None, None, :], 1 / 24)
+        assert np.array_equal(o_h[b], o_c[0]) and np.array_equal(l_h[b], l_c[0])
+    # (b) every position in order == dense
+    L = 129
+    allidx = np.arange(L)[None, None, :]
+    o_s, l_s = decode_sparse(q[1:], cache, bt[1:], np.array([L]), allidx, 1 / 24)
+    o_d, l_d = decode_dense(q[1:], cache, bt[1:], np.array([L]), 1 / 24, False)
+    assert np.array_equal(o_s, o_d) and np.array_equal(l_s, l_d)
+    # (c) order does not matter
+    sh = idx.copy()
+    for b in range(2):
+        rng.shuffle(sh[b, 0])
+    o1, l1 = decode_sparse(q, cache, bt, np.array(lens), idx, 1 / 24)
+    o2, l2 = decode_sparse(q, cache, bt, np.array(lens), sh, 1 / 24)
+    _close(o1, o2, 1e-13)
+    _close(l1, l2, 1e-13)
+
+
+def check_combine(attend, combine):
+    """Combining any split of the key set reproduces the unsplit result."""
+    rng = np.random.default_rng(13)
+    d_qk, d_v, T = 576, 512, 300
+    q = rng.standard_normal((4, d_qk))
+    k = rng.standard_normal((T, d_qk))
+    o_ref, l_ref = attend(q, k, 1 / 24, d_v)
+    for cuts in ([0, 1, T], [0, 64, 64, 200, T], [0, 150, 299, T]):   # includes an empty part
+        parts = [attend(q, k[a:b], 1 / 24, d_v) for a, b in zip(cuts[:-1], cuts[1:])]
+        o, l = combine(np.stack([p[0] for p in parts]), np.stack([p[1] for p in parts]))
+        _close(o, o_ref, 1e-13)
+        _close(l, l_ref, 1e-13)
+    o, l = combine(np.zeros((2, 4, d_v)), np.full((2, 4), -np.inf))
+    assert np.all(o == 0) and np.all(np.isneginf(l))
+
+
+def check_empty_key_sets(decode_dense, decode_sparse):
+    """Chosen reading for an empty key set: out 0, lse -inf."""
+    rng = np.random.default_rng(14)
+    d_qk = 576
+    cache, bt = _random_paged(rng, [64, 1], d_qk)
+    q = rng.standard_normal((2, 2, 2, d_qk))
+    out, lse = decode_dense(q, cache, bt, np.array([0, 1]), 1 / 24, True)
+    assert np.all(out[0] == 0) and np.all(np.isneginf(lse[0]))     # seqlen 0
+    assert np.all(out[1, 0] == 0) and np.all(np.isneginf(lse[1, 0]))  # causal row with no key
+    assert np.all(np.isfinite(lse[1, 1]))
+    idx = np.full((2, 2, 64), -1)
+    o, l = decode_sparse(q, cache, bt, np.array([64, 1]), idx, 1 / 24)
+    assert np.all(o == 0) and np.all(np.isneginf(l))
+
+
+def check_e4m3(e4m3_to_f64):
+    """All 256 codes vs torch's float8_e4m3fn decoding, plus closed forms."""
+    codes = np.arange(256, dtype=np.uint8)
+    mine = e4m3_to_f64(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    nan_m, nan_r = np.isnan(mine), np.isnan(ref)
+    assert np.array_equal(nan_m, nan_r)
+    assert np.array_equal(mine[~nan_m], ref[~nan_r])
+    fixed = {0x00: 0.0, 0x01: 2.0 ** -9, 0x07: 7 * 2.0 ** -9, 0x08: 2.0 ** -6, 0x38: 1.0,
+             0xB8: -1.0, 0x7E: 448.0, 0xFE: -448.0, 0x40: 2.0, 0x3C: 1.5}
+    for c, v in fixed.items():
+        assert e4m3_to_f64(np.array([c], dtype=np.uint8))[0] == v, hex(c)
+    assert np.isnan(e4m3_to_f64(np.array([0x7F, 0xFF], dtype=np.uint8))).all()
+
+
+def check_bf16_rounding(f32_round_to_bf16):
+    """fp32 -> bf16 round-to-nearest-even vs torch on random and tie values."""
+    rng = np.random.default_rng(15)
+    x = np.concatenate([rng.standard_normal(20000).astype(np.float32) * 10,
+                        np.array([1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -(1.0 + 2 ** -8),
+                                  3.0e38, 1e-40, 0.0, -0.0, 65504.0], dtype=np.float32)])
+    mine = f32_round_to_bf16(x)
+    ref = torch.from_numpy(x).to(torch.bfloat16).to(torch.float32).numpy()
+    assert np.array_equal(mine.view(np.uint32), ref.view(np.uint32))
+    assert f32_round_to_bf16(np.array([1.0 + 2 ** -8], np.float32))[0] == 1.0          # tie -> even
+    assert f32_round_to_bf16(np.array([1.0 + 3 * 2 ** -8], np.float32))[0] == 1.0 + 2 ** -6
+
+
+def check_fp8_record(dequant_fp8_records):
+    """A hand-built 656-byte record decodes to the hand-computed row."""
+    rec = np.zeros((1, PAGE, 656), dtype=np.uint8)
+    codes = np.array([0x38, 0xB8, 0x40, 0x7E], dtype=np.uint8)    # 1, -1, 2, 448
+    scales = np.array([0.5, 3.0, 1.0 / 448.0, 7.0], dtype=np.float32)
+    for t in range(4):
+        rec[0, t, :512] = codes[t]
+        rec[0, t, 512:528] = scales.view(np.uint8)
+        rope = np.full(64, t + 0.25, dtype=np.float32)
+        rec[0, t, 528:] = (rope.view(np.uint32) >> 16).astype(np.uint16).view(np.uint8)
+    out = dequant_fp8_records(rec)
+    vals = [1.0, -1.0, 2.0, 448.0]
+    for t in range(4):
+        for tile in range(4):
+            prod = np.float32(vals[t]) * scales[tile]
+            expect = float(torch.tensor(float(prod)).to(torch.bfloat16).float())
+            assert np.all(out[0, t, 128 * tile:128 * (tile + 1)] == expect), (t, tile)
+        assert np.all(out[0, t, 512:] == t + 0.25)
+
+
+def check_golden_two_tokens(decode_dense):
+    """Hand-derived closed form stored in tests/golden/two_token_closed_form.json."""
+    with open(os.path.join(GOLDEN, "two_token_closed_form.json")) as f:
+        g = json.load(f)
+    d = 576
+    cache = np.zeros((2, PAGE, d))
+    for t, row in enumerate(g["key_rows_sparse"]):
+        for k, v in row.items():
+            cache[1, t, int(k)] = v
+    q = np.zeros((1, 1, 1, d))
+    for k, v in g["q_sparse"].items():
+        q[0, 0, 0, int(k)] = v
+    bt = np.array([[1]])
+    out, lse = decode_dense(q, cache, bt, np.array([2]), g["scale"], False)
+    for k, v in g["out_sparse"].items():
+        _close(out[0, 0, 0, int(k)], v, 1e-15)
+    nz = set(int(k) for k in g["out_sparse"])
+    assert all(out[0, 0, 0, j] == 0 for j in range(512) if j not in nz)
+    _close(lse[0, 0, 0], g["lse"], 1e-15)

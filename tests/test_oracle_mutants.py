@@ -1,0 +1,149 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and check that at least
+one pin catches each of them. This shows the pins are tight enough that a
+dropped term, a wrong sign or index, or a transposed operand cannot pass."""
+import numpy as np
+import pytest
+
+from oracle import mla_oracle as O
+from tests import oracle_checks as C
+
+real_attend = O.attend
+
+
+def _attend_no_scale(q, k, scale, d_v=512):
+    return real_attend(q, k, 1.0, d_v)
+
+
+def _attend_neg(q, k, scale, d_v=512):
+    return real_attend(q, k, -scale, d_v)
+
+
+def _attend_shifted_v(q, k, scale, d_v=512):
+    q = np.asarray(q, float)
+    k = np.asarray(k, float)
+    if k.shape[0] == 0:
+        return np.zeros((q.shape[0], d_v)), np.full(q.shape[0], -np.inf)
+    s = scale * q @ k.T
+    m = s.max(1, keepdims=True)
+    e = np.exp(s - m)
+    v = np.roll(k, -1, axis=1)[:, :d_v]            # off-by-one value slice
+    return (e @ v) / e.sum(1, keepdims=True), (m + np.log(e.sum(1, keepdims=True)))[:, 0]
+
+
+def _attend_lse_is_max(q, k, scale, d_v=512):
+    o, l = real_attend(q, k, scale, d_v)
+    s = scale * np.asarray(q, float) @ np.asarray(k, float).T
+    return o, (s.max(1) if s.shape[1] else l)
+
+
+def _attend_log2(q, k, scale, d_v=512):
+    o, l = real_attend(q, k, scale, d_v)
+    return o, l / np.log(2.0)
+
+
+def _attend_unnormalised(q, k, scale, d_v=512):
+    o, l = real_attend(q, k, scale, d_v)
+    s = scale * np.asarray(q, float) @ np.asarray(k, float).T
+    if s.shape[1] == 0:
+        return o, l
+    return o * np.exp(s - s.max(1, keepdims=True)).sum(1, keepdims=True), l
+
+
+ATTEND_MUTANTS = [_attend_no_scale, _attend_neg, _attend_shifted_v, _attend_lse_is_max,
+                  _attend_log2, _attend_unnormalised]
+
+
+def _fails(fn, *a):
+    try:
+        fn(*a)
+    except AssertionError:
+        return True
+    return False
+
+
+@pytest.mark.parametrize("mutant", ATTEND_MUTANTS, ids=lambda f: f.__name__)
+def test_attend_mutants_caught(mutant, monkeypatch):
+    caught = _fails(C.check_brute_force_attend, mutant)
+    monkeypatch.setattr(O, "attend", mutant)
+    caught = caught or _fails(C.check_single_token, O.decode_dense)
+    caught = caught or _fails(C.check_lse_logsumexp, O.decode_dense)
+    assert caught
+
+
+def test_causal_off_by_one_caught(monkeypatch):
+    def decode_dense_bad(q, cache, bt, lens, scale, causal, d_v=512, requests=None):
+        # causal bound one token too short
+        if causal:
+            lens = np.asarray(lens)
+            q = np.asarray(q, float)
+            out, lse = O.decode_dense(q, cache, bt, lens, scale, False, d_v)
+            for b in range(q.shape[0]):
+                for i in range(q.shape[1]):
+                    n = max(0, min(int(lens[b]), int(lens[b]) - q.shape[1] + i))
+                    keys = O.gather_rows(cache, bt[b], np.arange(n))
+                    out[b, i], lse[b, i] = O.attend(q[b, i], keys, scale, d_v)
+            return out, lse
+        return O.decode_dense(q, cache, bt, lens, scale, causal, d_v)
+    assert _fails(C.check_brute_force_paged, decode_dense_bad, True)
+    assert _fails(C.check_causal_row0, decode_dense_bad)
+
+
+def test_page_lookup_mistake_caught(monkeypatch):
+    def gather_bad(cache, bt_row, positions):
+        positions = np.asarray(positions, dtype=np.int64)
+        pages = np.asarray(bt_row)[positions % len(bt_row)]        # wrong page index
+        return cache[pages, positions % 64]
+    monkeypatch.setattr(O, "gather_rows", gather_bad)
+    assert _fails(C.check_brute_force_paged, O.decode_dense, False)
+
+
+def test_sparse_minus_one_mistake_caught(monkeypatch):
+    def keys_bad(index_row, seqlen):
+        r = np.asarray(index_row, dtype=np.int64)
+        keep = r < seqlen                                   # -1 not excluded
+        return np.where(r[keep] < 0, seqlen - 1, r[keep]), np.array([], int), np.array([], int)
+    monkeypatch.setattr(O, "sparse_key_positions", keys_bad)
+    assert _fails(C.check_sparse, O.decode_sparse, O.decode_dense)
+
+
+def test_combine_mistake_caught():
+    def combine_bad(o_parts, lse_parts):
+        return np.asarray(o_parts).mean(0), np.asarray(lse_parts).max(0)
+    assert _fails(C.check_combine, O.attend, combine_bad)
+
+
+def test_e4m3_bias_mistake_caught():
+    def e4m3_bad(codes):
+        c = np.asarray(codes).astype(np.int64)
+        e = (c >> 3) & 0xF
+        m = c & 7
+        v = np.where(e == 0, m / 8.0 * 2.0 ** -7, (1 + m / 8.0) * np.exp2(e - 8.0))
+        return np.where(c & 0x80, -v, v)
+    assert _fails(C.check_e4m3, e4m3_bad)
+
+
+def test_bf16_truncation_caught():
+    def trunc(x):
+        x = np.ascontiguousarray(x, dtype=np.float32)
+        return (x.view(np.uint32) & np.uint32(0xFFFF0000)).view(np.float32)
+    assert _fails(C.check_bf16_rounding, trunc)
+
+
+def test_fp8_scale_tile_mistake_caught(monkeypatch):
+    monkeypatch.setattr(O, "FP8_TILE", 64)        # scales applied per 64 instead of 128
+    def deq(rec):
+        try:
+            return O.dequant_fp8_records(rec)
+        except ValueError:
+            raise AssertionError("shape")
+    assert _fails(C.check_fp8_record, deq)
+
+
+def test_value_slice_mistake_caught():
+    def decode_bad(q, cache, bt, lens, scale, causal, d_v=512, requests=None):
+        shifted = np.concatenate([cache[..., 64:], cache[..., :64]], axis=-1)  # V = dims 64..575
+        out, _ = O.decode_dense(q, shifted, bt, lens, scale, causal, d_v)
+        _, lse = O.decode_dense(q, cache, bt, lens, scale, causal, d_v)
+        return out, lse
+    assert _fails(C.check_single_token, decode_bad)
+    assert _fails(C.check_golden_two_tokens, decode_bad)

@@ -1,0 +1,62 @@
+"""The fp64 oracle against things other than itself (CPU only)."""
+import pytest
+
+from oracle import mla_oracle as O
+from tests import oracle_checks as C
+
+
+def test_brute_force_attend():
+    C.check_brute_force_attend(O.attend)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_brute_force_paged(causal):
+    C.check_brute_force_paged(O.decode_dense, causal)
+
+
+def test_single_token():
+    C.check_single_token(O.decode_dense)
+
+
+def test_constant_scores():
+    C.check_constant_scores(O.decode_dense)
+
+
+def test_lse_is_logsumexp():
+    C.check_lse_logsumexp(O.decode_dense)
+
+
+def test_page_permutation_invariance():
+    C.check_page_permutation(O.decode_dense)
+
+
+def test_causal_rows():
+    C.check_causal_row0(O.decode_dense)
+
+
+def test_sparse_rules():
+    C.check_sparse(O.decode_sparse, O.decode_dense)
+
+
+def test_combine_reproduces_unsplit():
+    C.check_combine(O.attend, O.combine)
+
+
+def test_empty_key_sets():
+    C.check_empty_key_sets(O.decode_dense, O.decode_sparse)
+
+
+def test_e4m3_all_codes():
+    C.check_e4m3(O.e4m3_to_f64)
+
+
+def test_bf16_rounding():
+    C.check_bf16_rounding(O.f32_round_to_bf16)
+
+
+def test_fp8_record_layout():
+    C.check_fp8_record(O.dequant_fp8_records)
+
+
+def test_golden_two_tokens():
+    C.check_golden_two_tokens(O.decode_dense)
