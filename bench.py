@@ -1,0 +1,388 @@
+#!/usr/bin/env python
+"""MLA paged decode benchmark (one JSON line on rank 0).
+
+A step is one pass of the whole decode path over one batch: split-KV
+scheduling (mla_get_metadata), the decode kernel and the split combine, all
+through the C ABI of libmla_b200.so on inputs already resident in HBM.
+Default workload: the DeepSeek-V3-shaped batch (64 requests x 128 heads,
+4096 cached tokens each, bf16 latent cache in 64-token pages), whose 302 MB
+cache is larger than L2, so no flush is needed between steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   # the fp64 CPU oracle, timed on host cores
+
+With N > 1 (launched by torch.distributed.run) every rank decodes its own
+replica of the workload (requests are independent; no collective is needed
+on the data path), timing is the max over ranks and `value` sums all ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import mla_workloads as W  # noqa: E402
+
+METRIC = "MLA decode TFLOPS & HBM GB/s on 1 B200, as fraction of roofline"
+PEAK_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAK_FALLBACK), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "head_latent_attention_get_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per decode launch from the committed ncu summary, if it was
+    taken on the current kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(workload)
+    if not e or e.get("kernel_source_sha") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+               "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, device, period_s: float = 0.002):
+        self.samples, self.reasons = [], set()
+        self.period = period_s
+        self.stop_evt = threading.Event()
+        self.ok = False
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+
+    def _run(self):
+        while not self.stop_evt.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self.stop_evt.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["nvml unavailable"]}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def workload_config(inp, work):
+    w = inp.workload
+    cfg = {"workload": f"{w.name}: {w.note}", "batch": w.batch, "s_q": w.s_q, "h_q": w.h_q,
+           "h_kv": 1, "d_qk": 576, "d_v": 512, "page": 64, "kv_cache": w.kv,
+           "causal": w.causal, "softmax_scale": w.scale,
+           "tokens_cached": int(sum(int(x) for x in inp.cache_seqlens.tolist())),
+           "algorithmic_flops": work["flops"], "algorithmic_bytes": work["bytes"],
+           "l2": "inputs larger than L2 (cache %.0f MB > 126 MB), no flush" % (
+               inp.kcache.numel() * inp.kcache.element_size() / 1e6)}
+    if w.topk:
+        cfg["topk"] = w.topk
+    return cfg
+
+
+# ----------------------------------------------------------------------------- oracle timing
+def oracle_sample(inp, budget_s: float):
+    """Time the fp64 oracle on whole requests until about budget_s elapses."""
+    from oracle import mla_oracle as O
+    from threadpoolctl import threadpool_info
+    w = inp.workload
+    order = list(range(w.batch))
+    flops = 0.0
+    elapsed = 0.0
+    done = []
+    for b in order:
+        sub = W.restrict(inp, [b])
+        work = W.algorithmic_work(sub)
+        t0 = time.perf_counter()
+        O.reference_decode(sub)
+        elapsed += time.perf_counter() - t0
+        flops += work["flops"]
+        done.append(b)
+        if elapsed >= budget_s:
+            break
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    return {"value": flops / elapsed / 1e12, "unit": "TFLOP/s", "cores": int(threads), "kind": "oracle",
+            "sample": f"{len(done)} of {w.batch} requests of the workload (whole requests, "
+                      f"{flops:.3g} FLOPs in {elapsed:.2f} s)"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    inp = W.make_inputs(W.get_workload(args.workload))
+    from oracle import mla_oracle as O
+    from threadpoolctl import threadpool_info
+    w = inp.workload
+    # each step decodes one request of the workload (a bounded sample)
+    times, flops = [], []
+    for s in range(args.warmup + args.steps):
+        b = s % w.batch
+        sub = W.restrict(inp, [b])
+        t0 = time.perf_counter()
+        O.reference_decode(sub)
+        dt = time.perf_counter() - t0
+        if s >= args.warmup:
+            times.append(dt)
+            flops.append(W.algorithmic_work(sub)["flops"])
+    tot = sum(times)
+    value = sum(flops) / tot / 1e12
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    work = W.algorithmic_work(inp)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / len(times),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(inp, work),
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": int(threads), "kind": "oracle",
+                             "sample": "one whole request of the workload per step"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- GPU path
+def run_gpu(args):
+    import head_latent_attention_get_b200 as M
+    from head_latent_attention_get_b200 import _capi as C
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        pg = dist
+
+    inp = W.make_inputs(W.get_workload(args.workload))
+    work = W.algorithmic_work(inp)
+    w = inp.workload
+    q = inp.q.to(dev)
+    kc = inp.kcache.to(dev)
+    bt = inp.block_table.to(dev)
+    sl = inp.cache_seqlens.to(dev)
+    idx = inp.indices.to(dev) if inp.indices is not None else None
+    runner = M.DecodeRunner(q, kc, bt, sl, softmax_scale=w.scale, causal=w.causal, indices=idx)
+    # timing variant: the decode kernel alone, then the combine enqueued by the caller
+    runner.args.debug_flags = C.MLA_DEBUG_SKIP_COMBINE
+    U, R, P = runner.units, runner.rows, runner.parts
+    ws_bytes = runner.workspace.numel()
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        runner.plan(stream)
+        if ev is not None:
+            ev[1].record(stream)
+        runner.run(stream)
+        if ev is not None:
+            ev[2].record(stream)
+        M.mla_combine(runner.workspace, ws_bytes, runner.num_splits, U, R, P, runner.out, runner.lse, stream)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    code, bits = runner.status()
+    if code != C.MLA_OK:
+        raise RuntimeError(f"device status after warm-up: {M.mla_status_string(code)} bits={bits}")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    bad_reasons = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
+    remeasured = False
+    for attempt in range(2):
+        if pg:
+            pg.barrier()
+        torch.cuda.synchronize()
+        with ClockSampler(dev) as clocks:
+            t_start.record(stream)
+            for s in range(args.steps):
+                step(evs[s])
+            t_end.record(stream)
+            torch.cuda.synchronize()
+        if pg:
+            pg.barrier()
+        if attempt == 0 and bad_reasons & set(clocks.summary().get("reasons", [])):
+            remeasured = True      # slowdown seen while timing: measure once more
+            continue
+        break
+    total_ms = t_start.elapsed_time(t_end)
+    meta_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    dec_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    comb_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    ms_step = total_ms / args.steps
+    if pg:
+        t = torch.tensor([ms_step], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms_step = float(t.item())
+
+    # ---- end to end through the public API with host buffers
+    q_h = inp.q.pin_memory()
+    bt_h = inp.block_table.pin_memory()
+    sl_h = inp.cache_seqlens.pin_memory()
+    idx_h = inp.indices.pin_memory() if inp.indices is not None else None
+    out_h = torch.empty(runner.out.shape, dtype=runner.out.dtype).pin_memory()
+    lse_h = torch.empty(runner.lse.shape, dtype=runner.lse.dtype).pin_memory()
+    runner_e2e = M.DecodeRunner(q, kc, bt, sl, softmax_scale=w.scale, causal=w.causal, indices=idx)
+
+    def e2e_step():
+        q.copy_(q_h, non_blocking=True)
+        bt.copy_(bt_h, non_blocking=True)
+        sl.copy_(sl_h, non_blocking=True)
+        if idx is not None:
+            idx.copy_(idx_h, non_blocking=True)
+        runner_e2e.plan(stream)
+        runner_e2e.run(stream)
+        out_h.copy_(runner_e2e.out, non_blocking=True)
+        lse_h.copy_(runner_e2e.lse, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    n_e2e = max(1, min(args.steps, 200))
+    e0.record(stream)
+    for _ in range(n_e2e):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / n_e2e
+    if pg:
+        t = torch.tensor([e2e_ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = q_h.numel() * q_h.element_size() + bt_h.numel() * 4 + sl_h.numel() * 4
+    if idx_h is not None:
+        h2d += idx_h.numel() * 4
+    d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * 4
+
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peaks, peak_src = load_peaks()
+    hbm_peak = float(peaks["hbm_gbs"])
+    tc_peak = float(peaks["bf16_tflops"])
+    dec_avg = sum(dec_ms) / len(dec_ms)
+    achieved_gbs = work["bytes"] / (dec_avg * 1e-3) / 1e9
+    achieved_tf = work["flops"] / (dec_avg * 1e-3) / 1e12
+    t_hbm = work["bytes"] / (hbm_peak * 1e9)
+    t_tc = work["flops"] / (tc_peak * 1e12)
+    bound = "hbm" if t_hbm >= t_tc else "tensor"
+    traffic = recorded_traffic(w.name)
+    roof = {"bound": bound,
+            "achieved": achieved_gbs if bound == "hbm" else achieved_tf,
+            "peak": hbm_peak if bound == "hbm" else tc_peak,
+            "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
+            "frac": (achieved_gbs / hbm_peak) if bound == "hbm" else (achieved_tf / tc_peak),
+            "traffic": traffic,
+            "peak_source": f"{peak_src} (MEASURED_PEAKS.json burst figures)" if peak_src == "measured"
+            else "fallback",
+            "kernel": "mla_decode_kernel",
+            "kernel_ms": dec_avg,
+            "hbm_frac": achieved_gbs / hbm_peak, "tensor_frac": achieved_tf / tc_peak,
+            "roofline_frac": max(t_hbm, t_tc) / (dec_avg * 1e-3),
+            "combine_ms": sum(comb_ms) / len(comb_ms), "metadata_ms": sum(meta_ms) / len(meta_ms)}
+    value = world * work["flops"] / (ms_step * 1e-3) / 1e12
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if w.kv == "bf16" else "fp8-e4m3 cache, bf16 mma",
+            "data": "synthetic", "config": workload_config(inp, work),
+            "hbm_gbs": world * work["bytes"] / (ms_step * 1e-3) / 1e9,
+            "roofline": roof, "clocks": dict(clocks.summary(), remeasured=remeasured),
+            "e2e": {"value": world * work["flops"] / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": 3 * args.steps}
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_sample(inp, args.cpu_budget)
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="dsv3", choices=[w.name for w in W.named_workloads()])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)   # at least 3 untimed warm-up steps
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,39 @@
+// Kernel parameter block and launchers shared by the host API and the kernels.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "mla_common.cuh"
+
+namespace mla {
+
+enum KvMode : int { kModeBf16 = 0, kModeFp8 = 1, kModeSparse = 2 };
+
+struct DecodeParams {
+  int units, rows, h_q, s_q, causal, topk;  // rows = query rows per unit
+  float scale, scale_log2;                  // softmax scale, and scale * log2(e)
+  int num_pages, bt_stride;
+  const int32_t* block_table;
+  const int32_t* seqlens;
+  const int32_t* indices;                   // sparse mode
+  const uint8_t* kcache_fp8;                // FP8 mode: token records
+  const int32_t* tile_md;
+  const int32_t* split_ptr;
+  void* out;                                // bf16 [units*rows][512]
+  float* lse;                               // [units*rows]
+  float* ws_lse;                            // workspace partial LSE
+  float* ws_o;                              // workspace partial O
+  uint32_t* status;                         // device status word
+  uint64_t timeout_ns;
+  uint32_t debug_flags;
+};
+
+cudaError_t launch_decode(int rows_per_cta, int mode, const CUtensorMap& tq, const CUtensorMap& tkv,
+                          const CUtensorMap& taux, const DecodeParams& p, int parts, int row_groups,
+                          cudaStream_t stream);
+mla_status_t launch_metadata(const int32_t* seqlens, int U, int topk, int parts, int32_t* tile_md,
+                             int32_t* num_splits, cudaStream_t stream);
+mla_status_t launch_combine(const void* workspace, int units, int rows, int parts, const int32_t* split_ptr,
+                            void* out, float* lse, cudaStream_t stream);
+
+}  // namespace mla

@@ -1,0 +1,193 @@
+// Split-KV tile scheduler ("get_mla_metadata": "Qu'est-ce que FlashMLA ?",
+// section "Obtenir les métadonnées MLA" — computed once per decode step from
+// cache_seqlens and reused by every layer).
+//
+// Every work unit (a request for paged decoding, a (request, query token)
+// pair for sparse decoding) costs n_u tiles of 128 tokens plus a fixed
+// overhead of kSchedOverhead tiles (loading Q, writing a partial result,
+// combining). Units are laid end to end on a cost axis [0, total); part p
+// takes the cost range [p*payload, (p+1)*payload) with payload =
+// ceil(total / parts). Tile k of unit u sits at cost position
+// C_u + overhead + k, so it belongs to part floor(position / payload): every
+// tile lands in exactly one part, parts are contiguous in (unit, tile)
+// order, and the number of parts touching unit u follows in closed form.
+// The cost axis is int32 (the prefix is stored in num_splits), so the sum of
+// all tile counts plus overheads must stay below 2^31.
+#include <cuda_runtime.h>
+
+#include "mla_kernels.cuh"
+
+namespace mla {
+
+__host__ __device__ inline int unit_tiles(const int32_t* seqlens, int u, int topk) {
+  if (topk > 0) return (topk + kTile - 1) / kTile;
+  int L = seqlens[u];
+  return L > 0 ? (L + kTile - 1) / kTile : 0;
+}
+
+// position on the cost axis -> {unit, tile} of the first tile at or after it
+__host__ __device__ inline int2 cost_to_tile(const int32_t* C, int U, int total, int x) {
+  if (x >= total) return make_int2(U, 0);
+  int lo = 0, hi = U - 1;  // last u with C[u] <= x (C non-decreasing, C[0] = 0)
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (C[mid] <= x) lo = mid; else hi = mid - 1;
+  }
+  // zero-cost units share C with the next unit; the binary search lands on the
+  // last unit with C[u] <= x, which is the one whose cost range contains x.
+  const int local = x - C[lo] - kSchedOverhead;
+  return make_int2(lo, local > 0 ? (int)local : 0);
+}
+
+__host__ __device__ inline int first_part_of(int Cu, int payload) {
+  return (int)((Cu + kSchedOverhead) / payload);
+}
+
+// ---------------------------------------------------------------- host twin
+extern "C" mla_status_t mla_get_metadata_host(const int32_t* cache_seqlens, int batch, int s_q, int h_q,
+                                              int h_kv, int topk, int num_sm_parts, int32_t* tile_md,
+                                              int32_t* num_splits) {
+  if (!tile_md || !num_splits || batch <= 0 || s_q <= 0 || h_q <= 0 || h_kv <= 0 || num_sm_parts <= 0)
+    return MLA_ERR_INVALID_ARG;
+  if (topk < 0 || (topk > 0 && topk % 64 != 0)) return MLA_ERR_INVALID_ARG;
+  if (topk == 0 && !cache_seqlens) return MLA_ERR_INVALID_ARG;
+  if (h_kv != 1) return MLA_ERR_UNSUPPORTED;
+  const int U = topk > 0 ? batch * s_q : batch;
+  // cost prefix C[0..U] kept in num_splits first, then replaced by split pointers
+  int total = 0;
+  for (int u = 0; u < U; ++u) {
+    num_splits[u] = (int32_t)total;
+    int n = unit_tiles(cache_seqlens, u, topk);
+    total += n > 0 ? n + kSchedOverhead : 0;
+  }
+  num_splits[U] = (int32_t)total;
+  const int payload = total > 0 ? (total + num_sm_parts - 1) / num_sm_parts : 1;
+  for (int p = 0; p < num_sm_parts; ++p) {
+    const int2 b = cost_to_tile(num_splits, U, total, p * payload);
+    const int2 e = cost_to_tile(num_splits, U, total, (p + 1) * payload);
+    int32_t* md = tile_md + p * MLA_TILE_MD_INTS;
+    md[0] = b.x; md[1] = b.y; md[2] = e.x; md[3] = e.y;
+    md[4] = b.x < U ? p - first_part_of(num_splits[b.x], payload) : 0;
+    md[5] = (int32_t)payload; md[6] = 0; md[7] = 0;
+  }
+  int32_t acc = 0;
+  for (int u = 0; u < U; ++u) {
+    const int Cu = num_splits[u];
+    const int n = unit_tiles(cache_seqlens, u, topk);
+    int ns = 0;
+    if (n > 0) ns = (int)((Cu + kSchedOverhead + n - 1) / payload) - first_part_of(Cu, payload) + 1;
+    num_splits[u] = acc;
+    acc += ns;
+  }
+  num_splits[U] = acc;
+  for (int p = 0; p < num_sm_parts; ++p) {
+    int32_t* md = tile_md + p * MLA_TILE_MD_INTS;
+    if (md[0] < U) md[4] += num_splits[md[0]];
+  }
+  return MLA_OK;
+}
+
+// ---------------------------------------------------------------- device kernel
+constexpr int kMetaThreads = 256;
+
+// returns {exclusive prefix of v over the block, block total}
+__device__ int2 block_exclusive_scan(int v) {
+  __shared__ int warp_sums[kMetaThreads / 32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_sums[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < kMetaThreads / 32 ? warp_sums[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    if (lane < kMetaThreads / 32) warp_sums[lane] = w;  // inclusive
+  }
+  __syncthreads();
+  const int before = (warp > 0 ? warp_sums[warp - 1] : 0) + x - v;
+  const int total = warp_sums[kMetaThreads / 32 - 1];
+  __syncthreads();
+  return make_int2(before, total);
+}
+
+__global__ void __launch_bounds__(kMetaThreads) mla_metadata_kernel(const int32_t* __restrict__ seqlens,
+                                                                   int U, int topk, int parts,
+                                                                   int32_t* __restrict__ tile_md,
+                                                                   int32_t* __restrict__ num_splits) {
+  __shared__ int s_payload;
+  const int t = threadIdx.x;
+  const int per = (U + kMetaThreads - 1) / kMetaThreads;
+  const int u0 = min(U, t * per), u1 = min(U, u0 + per);
+  // 1. cost prefix C[u] -> num_splits[u], total -> num_splits[U]
+  int my = 0;
+  for (int u = u0; u < u1; ++u) {
+    int n = unit_tiles(seqlens, u, topk);
+    my += n > 0 ? n + kSchedOverhead : 0;
+  }
+  const int2 sc = block_exclusive_scan(my);
+  const int total = sc.y;
+  int c = sc.x;
+  for (int u = u0; u < u1; ++u) {
+    num_splits[u] = c;
+    int n = unit_tiles(seqlens, u, topk);
+    c += n > 0 ? n + kSchedOverhead : 0;
+  }
+  if (t == 0) {
+    num_splits[U] = total;
+    s_payload = total > 0 ? (total + parts - 1) / parts : 1;
+  }
+  __syncthreads();
+  const int payload = s_payload;
+  // 2. part boundaries (binary search on C)
+  for (int p = t; p < parts; p += kMetaThreads) {
+    const int2 b = cost_to_tile(num_splits, U, total, p * payload);
+    const int2 e = cost_to_tile(num_splits, U, total, (p + 1) * payload);
+    int32_t* md = tile_md + p * MLA_TILE_MD_INTS;
+    md[0] = b.x; md[1] = b.y; md[2] = e.x; md[3] = e.y;
+    md[4] = b.x < U ? p - first_part_of(num_splits[b.x], payload) : 0;
+    md[5] = (int32_t)payload; md[6] = 0; md[7] = 0;
+  }
+  __syncthreads();
+  // 3. splits per unit -> exclusive prefix in num_splits
+  int mys = 0;
+  for (int u = u0; u < u1; ++u) {
+    const int Cu = num_splits[u];
+    const int n = unit_tiles(seqlens, u, topk);
+    if (n > 0) mys += (int)((Cu + kSchedOverhead + n - 1) / payload) - first_part_of(Cu, payload) + 1;
+  }
+  const int2 ss = block_exclusive_scan(mys);
+  const int tot_splits = ss.y;
+  int sp = ss.x;
+  for (int u = u0; u < u1; ++u) {
+    const int Cu = num_splits[u];  // read before overwriting this slot
+    const int n = unit_tiles(seqlens, u, topk);
+    int ns = 0;
+    if (n > 0) ns = (int)((Cu + kSchedOverhead + n - 1) / payload) - first_part_of(Cu, payload) + 1;
+    num_splits[u] = sp;
+    sp += ns;
+  }
+  __syncthreads();
+  if (t == 0) num_splits[U] = tot_splits;
+  __syncthreads();
+  // 4. workspace index of each part's first piece
+  for (int p = t; p < parts; p += kMetaThreads) {
+    int32_t* md = tile_md + p * MLA_TILE_MD_INTS;
+    if (md[0] < U) md[4] += num_splits[md[0]];
+  }
+}
+
+mla_status_t launch_metadata(const int32_t* seqlens, int U, int topk, int parts, int32_t* tile_md,
+                             int32_t* num_splits, cudaStream_t stream) {
+  mla_metadata_kernel<<<1, kMetaThreads, 0, stream>>>(seqlens, U, topk, parts, tile_md, num_splits);
+  return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+}  // namespace mla

@@ -1,0 +1,223 @@
+/*
+ * mla.h — C ABI of a B200 (sm_100a) library for Multi-head Latent Attention
+ * (MLA) decoding over a paged latent KV cache.
+ *
+ * What the library computes (for request b, query token i < s_q, head h):
+ *   s_t  = softmax_scale * <q[b,i,h,0:576], row(t)[0:576]>      (K = whole row)
+ *   out  = sum_t softmax(s)_t * row(t)[0:512]                    (V = first 512)
+ *   lse  = ln sum_t exp(s_t)                                     (natural log)
+ * over the key set t of the request: all cached tokens (t < cache_seqlens[b]),
+ * restricted by the causal mask t <= seqlen - s_q + i when `causal` is set,
+ * or, for sparse decoding, the token positions listed in `indices[b,i,:]`
+ * (entries equal to -1 are ignored). An empty key set gives out = 0 and
+ * lse = -inf.
+ *
+ * Sources (web pages on FlashMLA):
+ *   - "Qu'est-ce que FlashMLA ?" (topnet.top), sections "Obtenir les
+ *     métadonnées MLA" and "Exécuter le décodage MLA": the two-call shape
+ *     get_mla_metadata(cache_seqlens, s_q*h_q//h_kv, h_kv) ->
+ *     (tile_scheduler_metadata, num_splits), computed once per decode step
+ *     and reused by every layer's flash_mla_with_kvcache(q, kvcache,
+ *     block_table, cache_seqlens, dv, metadata, num_splits, causal).
+ *   - "DeepSeek, FlashMLA 오픈소스 공개" (GeekNews), Summary: BF16, paged
+ *     KV cache with block size 64, variable-length serving.
+ *   - "[flashinfer] FlashInfer, NVFP4를 활용한 DeepSeek-V4 디코딩 성능 최적화",
+ *     section 2 (nvfp4_mla_decode README): one latent row per token is both
+ *     K and V; 64-token pages; causal mask inside the query block against the
+ *     request's last tokens; BF16 out and natural-log FP32 LSE; tensor table
+ *     (block_tables [batch, max_pages] int32, seq_lens [batch] int32);
+ *     caller-owned workspace buffer; section 3: split-KV combine kernel.
+ *   - deepseek-ai/FlashMLA (agentlenshq), "기술적 세부 사항": FP8 latent
+ *     cache stores quantised values plus scale factors dequantised on the
+ *     fly; sparse decoding takes an indices tensor whose -1 entries are
+ *     ignored.
+ *
+ * Conventions for every entry point:
+ *   - Pointers documented "device" must point to memory of the current CUDA
+ *     device; "host" pointers to host memory. The caller owns every buffer;
+ *     the library allocates no memory and keeps no per-call state.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL = the
+ *     legacy default stream). Host-side argument checks run synchronously
+ *     before any launch and return an error code without launching.
+ *   - Device-side problems (a page id outside [0, num_pages), a request longer
+ *     than its block-table row, a wait that exceeded its time limit) never
+ *     trap: the kernel skips the bad item and ORs a bit into a status word
+ *     kept in the workspace; read it with mla_query_device_status().
+ *   - Only h_kv == 1 (the MLA latent cache), d_qk == 576, d_v == 512 and a
+ *     page size of 64 are implemented.
+ */
+#ifndef MLA_B200_H_
+#define MLA_B200_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* mla_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARG = 1,         /* null/misaligned pointer, bad size or shape */
+  MLA_ERR_UNSUPPORTED = 2,         /* valid request outside what is implemented */
+  MLA_ERR_WORKSPACE_TOO_SMALL = 3, /* workspace_bytes < mla_workspace_size(...) */
+  MLA_ERR_CUDA = 4,                /* a CUDA runtime/driver call failed */
+  MLA_ERR_DEVICE_TIMEOUT = 5,      /* status word: a device wait hit its limit */
+  MLA_ERR_DEVICE_BOUNDS = 6        /* status word: an index/page was out of range */
+} mla_status_t;
+
+/* KV cache storage formats (mla_decode_args.kv_format). */
+enum {
+  /* bf16 [num_pages, 64, 1, 576]; token row = 512 latent + 64 RoPE dims. */
+  MLA_KV_BF16 = 0,
+  /* uint8 [num_pages, 64, 656] token records, byte layout
+   *   [0,512)   512 e4m3 latent codes (OCP FP8 E4M3, no infinities)
+   *   [512,528) 4 fp32 scales, scale k applies to latent dims [128k,128k+128)
+   *   [528,656) 64 bf16 RoPE dims
+   * dequantised value = bf16_rne(fp32(e4m3) * scale), product rounded to
+   * nearest in fp32; the RoPE dims are used as stored. */
+  MLA_KV_FP8_E4M3 = 1
+};
+
+/* Bits of the device status word kept at the start of the workspace. */
+enum {
+  MLA_DEVICE_STATUS_TIMEOUT = 1u, /* an mbarrier wait exceeded timeout_ns */
+  MLA_DEVICE_STATUS_BOUNDS = 2u   /* page id, block-table slot or index out of range */
+};
+
+/* Test and timing hooks for mla_decode_args.debug_flags (0 in normal use). */
+enum {
+  /* The MMA issuer withholds its first "scores ready" signal, so the
+   * softmax warps' bounded wait runs out: exercises the timeout path. */
+  MLA_DEBUG_WITHHOLD_SCORES = 1u,
+  /* mla_decode_* enqueue only the decode kernel; the caller enqueues
+   * mla_combine afterwards (lets a profiler or timer separate the two). */
+  MLA_DEBUG_SKIP_COMBINE = 2u
+};
+
+#define MLA_D_QK 576
+#define MLA_D_V 512
+#define MLA_PAGE_SIZE 64
+#define MLA_TILE_MD_INTS 8 /* int32 entries per scheduler part */
+#define MLA_MAX_ROWS 128   /* max query rows (s_q*h_q/h_kv, or h_q when sparse) */
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* mla_status_string(mla_status_t status);
+
+/* Number of scheduler parts for a problem on `device` (host-only query).
+ * rows = s_q*h_q/h_kv for paged decoding, h_q for sparse decoding
+ * (topk > 0). One part is processed by ceil(rows/64) CTAs, one per SM, so
+ * parts = floor(num_SMs / ceil(rows/64)). Writes *num_sm_parts. */
+mla_status_t mla_get_num_sm_parts(int device, int s_q, int h_q, int h_kv, int topk, int* num_sm_parts);
+
+/* Split-KV tile scheduler ("get_mla_metadata" in the pages' API).
+ *
+ * Work units: paged decoding (topk == 0) has one unit per request b with
+ * ceil(cache_seqlens[b]/128) blocks of 128 tokens (two pages); sparse
+ * decoding (topk > 0) has one unit per (b, i), i < s_q, with ceil(topk/128)
+ * blocks of 128 index slots. Every unit costs its blocks plus a fixed
+ * overhead of 3 blocks; the units are laid end to end and cut into
+ * num_sm_parts ranges of equal cost, so one part covers a contiguous run of
+ * (unit, block) pairs and a unit may be split across parts. The total cost
+ * must stay below 2^31.
+ *
+ *   cache_seqlens  device int32 [batch]; read only when topk == 0 (may be
+ *                  NULL when topk > 0).
+ *   tile_md        device int32 [num_sm_parts * MLA_TILE_MD_INTS], written:
+ *                  per part {begin_unit, begin_block, end_unit, end_block
+ *                  (exclusive, lexicographic), workspace index of the
+ *                  part's first piece, cost per part, 0, 0}.
+ *   num_splits     device int32 [units + 1], written: exclusive prefix sum
+ *                  of the number of parts touching each unit (a unit with
+ *                  no blocks has 0 splits).
+ * Both outputs are reusable by every layer of the same decode step.
+ * Errors: INVALID_ARG for null outputs or non-positive sizes, topk % 64 != 0;
+ * UNSUPPORTED for h_kv != 1. */
+mla_status_t mla_get_metadata(const int32_t* cache_seqlens, int batch, int s_q, int h_q, int h_kv,
+                              int topk, int num_sm_parts, int32_t* tile_md, int32_t* num_splits,
+                              mla_stream_t stream);
+
+/* The same scheduler run on the host: all pointers are host pointers and the
+ * call is synchronous. Produces exactly what mla_get_metadata produces. */
+mla_status_t mla_get_metadata_host(const int32_t* cache_seqlens, int batch, int s_q, int h_q, int h_kv,
+                                   int topk, int num_sm_parts, int32_t* tile_md, int32_t* num_splits);
+
+/* Bytes of caller-owned workspace a decode call needs:
+ *   256-byte header (the device status word at offset 0), then
+ *   partial LSE  fp32 [units + num_sm_parts][rows]          (256-B aligned)
+ *   partial O    fp32 [units + num_sm_parts][rows][512]     (256-B aligned)
+ * Split s of unit u is entry num_splits[u] + s of the partial arrays; each
+ * partial O is already divided by its own softmax denominator. Returns 0 for
+ * invalid sizes. A fresh workspace must have its status word cleared once
+ * (mla_clear_device_status) before its first use. */
+size_t mla_workspace_size(int batch, int s_q, int h_q, int h_kv, int topk, int num_sm_parts);
+
+typedef struct {
+  const void* q;                /* device bf16 [batch, s_q, h_q, 576], 16-B aligned */
+  const void* kcache;           /* device, format per kv_format, 16-B aligned */
+  const int32_t* block_table;   /* device int32 [batch, block_table_stride]; entry
+                                   j of row b = physical page of tokens [64j, 64j+64) */
+  const int32_t* cache_seqlens; /* device int32 [batch] */
+  const int32_t* tile_md;       /* device, from mla_get_metadata (same sizes) */
+  const int32_t* num_splits;    /* device, from mla_get_metadata */
+  void* out;                    /* device bf16 [batch, s_q, h_q, 512], written */
+  float* lse;                   /* device fp32 [batch, s_q, h_q], written */
+  void* workspace;              /* device, >= mla_workspace_size(...) bytes */
+  size_t workspace_bytes;
+  int batch, s_q, h_q, h_kv;
+  int d_qk, d_v;                /* must be 576 and 512 */
+  int page_size;                /* must be 64 */
+  int num_pages;                /* physical pages in kcache */
+  int block_table_stride;       /* int32 elements between block-table rows */
+  int num_sm_parts;             /* the value passed to mla_get_metadata */
+  float softmax_scale;          /* multiplies q.k before the softmax */
+  int causal;                   /* nonzero: causal mask inside the s_q block */
+  int kv_format;                /* MLA_KV_BF16 or MLA_KV_FP8_E4M3 */
+  uint64_t timeout_ns;          /* limit of every device wait; 0 = 2 s */
+  uint32_t debug_flags;         /* MLA_DEBUG_* test hooks; 0 normally */
+} mla_decode_args;
+
+/* Paged decoding: enqueues the decode kernel and the split combine.
+ * Output rows of units processed in one piece are written by the decode
+ * kernel; split units and empty units are finished by the combine. Errors:
+ * INVALID_ARG (null or misaligned pointers, d_qk/d_v/page_size mismatch,
+ * non-positive sizes, bad kv_format), UNSUPPORTED (h_kv != 1, rows >
+ * MLA_MAX_ROWS), WORKSPACE_TOO_SMALL, CUDA (launch failure). */
+mla_status_t mla_decode_paged(const mla_decode_args* args, mla_stream_t stream);
+
+/* Token-sparse decoding. indices: device int32 [batch, s_q, topk], logical
+ * token positions of request b resolved through its block-table row; -1
+ * entries are ignored; other values outside [0, cache_seqlens[b]) are ignored
+ * and set MLA_DEVICE_STATUS_BOUNDS; duplicates count as often as they occur.
+ * topk must be a positive multiple of 64; `causal` is ignored; kv_format must
+ * be MLA_KV_BF16. tile_md/num_splits come from mla_get_metadata(..., topk).
+ * Errors as for mla_decode_paged. */
+mla_status_t mla_decode_sparse(const mla_decode_args* args, const int32_t* indices, int topk,
+                               mla_stream_t stream);
+
+/* Split-KV combine alone (mla_decode_* call it already). For every unit u
+ * with n = num_splits[u+1] - num_splits[u]:
+ *   n >= 2: lse = ln sum_s exp(lse_s), out = sum_s exp(lse_s - lse) * o_s
+ *           over the workspace partials (fp32), out rounded to bf16;
+ *   n == 0: out = 0, lse = -inf;   n == 1: nothing is written.
+ * out/lse rows of unit u start at row u*rows_per_unit (rows = s_q*h_q for
+ * paged units, h_q for sparse units; see mla_workspace_size). */
+mla_status_t mla_combine(const void* workspace, size_t workspace_bytes, const int32_t* num_splits,
+                         int num_units, int rows_per_unit, int num_sm_parts, void* out, float* lse,
+                         mla_stream_t stream);
+
+/* Reads the device status word (blocks until `stream` reaches this point).
+ * Returns MLA_OK, MLA_ERR_DEVICE_TIMEOUT or MLA_ERR_DEVICE_BOUNDS (timeout
+ * wins when both are set) and stores the raw bits in *status_bits when
+ * status_bits is not NULL. The word stays set until cleared. */
+mla_status_t mla_query_device_status(const void* workspace, uint32_t* status_bits, mla_stream_t stream);
+
+/* Zeroes the device status word (asynchronous on `stream`). */
+mla_status_t mla_clear_device_status(void* workspace, mla_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MLA_B200_H_ */

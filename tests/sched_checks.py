@@ -1,0 +1,70 @@
+"""Invariants of the split-KV tile scheduler output.
+
+Any exact cover is a valid schedule, so these checks test properties, not
+bytes: every (unit, tile) pair lands in exactly one part, parts are
+contiguous, the split counts match the parts that touch each unit, each
+piece's workspace slot is unique within its unit, and no part carries much
+more than its share of the cost.
+"""
+import numpy as np
+
+TILE = 128
+OVERHEAD = 3
+
+
+def unit_tiles(seqlens, batch, s_q, topk):
+    if topk:
+        return [(topk + TILE - 1) // TILE] * (batch * s_q)
+    return [max(0, (int(L) + TILE - 1) // TILE) for L in seqlens[:batch]]
+
+
+def pieces_of_part(md, n):
+    bu, bt, eu, et, first_ws = (int(x) for x in md[:5])
+    out = []
+    u, t, first = bu, bt, True
+    U = len(n)
+    while u < U and (u < eu or (u == eu and t < et)):
+        tend = min(et, n[u]) if u == eu else n[u]
+        if t < tend:
+            out.append((u, t, tend, first))
+        first = False
+        u, t = u + 1, 0
+    return out
+
+
+def check_schedule(tile_md, num_splits, seqlens, batch, s_q, topk, parts):
+    n = unit_tiles(seqlens, batch, s_q, topk)
+    U = len(n)
+    md = np.asarray(tile_md).reshape(parts, 8)
+    ptr = np.asarray(num_splits)[:U + 1]
+    assert ptr[0] == 0 and np.all(np.diff(ptr) >= 0)
+    seen = {}
+    touch = [[] for _ in range(U)]
+    cost = []
+    for p in range(parts):
+        pcs = pieces_of_part(md[p], n)
+        c = 0
+        for (u, t0, t1, first) in pcs:
+            for k in range(t0, t1):
+                assert (u, k) not in seen, f"tile {(u, k)} in parts {seen[(u, k)]} and {p}"
+                seen[(u, k)] = p
+            touch[u].append((p, t0, first))
+            c += (t1 - t0) + OVERHEAD
+        cost.append(c)
+    expected = {(u, k) for u in range(U) for k in range(n[u])}
+    assert set(seen) == expected, "schedule does not cover every tile exactly once"
+    for u in range(U):
+        ns = len(touch[u])
+        assert ptr[u + 1] - ptr[u] == ns, (u, ptr[u + 1] - ptr[u], ns)
+        # the first piece of a unit starts at tile 0, later pieces continue it
+        ts = [t0 for (_, t0, _) in touch[u]]
+        assert ts == sorted(ts) and (not ts or ts[0] == 0)
+        for j, (p, t0, first) in enumerate(touch[u]):
+            if ns >= 2:
+                ws = int(md[p][4]) if first else int(ptr[u])
+                assert ws == ptr[u] + j, (u, p, ws, ptr[u] + j)
+    assert ptr[U] <= U + parts
+    total = sum(x + OVERHEAD for x in n if x > 0)
+    payload = -(-total // parts) if total else 1
+    assert max(cost) <= payload + 2 * OVERHEAD, (max(cost), payload)
+    return {"payload": payload, "max_cost": max(cost), "splits": int(ptr[U])}

@@ -1,0 +1,146 @@
+"""The C-ABI library on the host: it loads, exports every declared entry
+point, and rejects bad arguments before launching anything (CPU only)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import head_latent_attention_get_b200 as M
+from head_latent_attention_get_b200 import _capi as C
+from tests import sched_checks as S
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = []
+    for f in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if f.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", f)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"\b(mla_[a-z0-9_]+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_library_exports_every_declared_function():
+    names = declared_functions()
+    assert "mla_decode_paged" in names and "mla_get_metadata" in names and len(names) >= 10
+    L = C.lib()
+    missing = [n for n in names if not hasattr(L, n)]
+    assert not missing, missing
+
+
+def test_status_strings():
+    for code in range(7):
+        assert M.mla_status_string(code).startswith("MLA_")
+    assert M.mla_status_string(99) == "MLA_ERR_UNKNOWN"
+
+
+def test_workspace_size_layout():
+    # header 256 + lse [(U+P) x R] f32 (256-aligned) + o [(U+P) x R x 512] f32
+    U, R, P = 64, 128, 74
+    lse = (U + P) * R * 4
+    o_off = -(-(256 + lse) // 256) * 256
+    total = -(-(o_off + (U + P) * R * 512 * 4) // 256) * 256
+    assert M.mla_workspace_size(64, 1, 128, 1, 0, 74) == total
+    assert M.mla_workspace_size(32, 1, 128, 1, 2048, 74) == M.mla_workspace_size(32, 1, 128, 1, 0, 74)
+    assert M.mla_workspace_size(0, 1, 16, 1, 0, 10) == 0
+
+
+def _fake_args(**over):
+    # non-null, 16-byte aligned fake device pointers: only host checks run
+    base = dict(q=None, kcache=None, block_table=None, cache_seqlens=None, tile_md=None, num_splits=None,
+                out=None, lse=None, workspace=None)
+    a = C.MlaDecodeArgs()
+    for i, k in enumerate(base):
+        setattr(a, k, 0x100000 * (i + 1))
+    a.workspace_bytes = 1 << 40
+    a.batch, a.s_q, a.h_q, a.h_kv = 2, 1, 16, 1
+    a.d_qk, a.d_v, a.page_size = 576, 512, 64
+    a.num_pages, a.block_table_stride, a.num_sm_parts = 8, 4, 148
+    a.softmax_scale, a.causal, a.kv_format = 1 / 24, 0, C.MLA_KV_BF16
+    for k, v in over.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(q=None), C.MLA_ERR_INVALID_ARG),
+    (dict(out=0x100008), C.MLA_ERR_INVALID_ARG),              # misaligned
+    (dict(d_qk=512), C.MLA_ERR_INVALID_ARG),
+    (dict(d_v=576), C.MLA_ERR_INVALID_ARG),
+    (dict(page_size=128), C.MLA_ERR_INVALID_ARG),
+    (dict(batch=0), C.MLA_ERR_INVALID_ARG),
+    (dict(kv_format=7), C.MLA_ERR_INVALID_ARG),
+    (dict(softmax_scale=float("nan")), C.MLA_ERR_INVALID_ARG),
+    (dict(h_kv=2, h_q=32), C.MLA_ERR_UNSUPPORTED),
+    (dict(h_q=256), C.MLA_ERR_UNSUPPORTED),
+    (dict(s_q=2, h_q=128), C.MLA_ERR_UNSUPPORTED),
+    (dict(workspace_bytes=1024), C.MLA_ERR_WORKSPACE_TOO_SMALL),
+])
+def test_decode_rejects_bad_arguments(over, code):
+    a = _fake_args(**over)
+    assert C.lib().mla_decode_paged(ctypes.byref(a), None) == code
+
+
+def test_sparse_rejects_bad_topk_and_fp8():
+    a = _fake_args()
+    L = C.lib()
+    assert L.mla_decode_sparse(ctypes.byref(a), 0x200000, 100, None) == C.MLA_ERR_INVALID_ARG
+    assert L.mla_decode_sparse(ctypes.byref(a), None, 128, None) == C.MLA_ERR_INVALID_ARG
+    a8 = _fake_args(kv_format=C.MLA_KV_FP8_E4M3)
+    assert L.mla_decode_sparse(ctypes.byref(a8), 0x200000, 128, None) == C.MLA_ERR_UNSUPPORTED
+    assert L.mla_decode_paged(None, None) == C.MLA_ERR_INVALID_ARG
+
+
+def test_metadata_rejects_bad_arguments():
+    L = C.lib()
+    assert L.mla_get_metadata(0x1000, 2, 1, 16, 1, 0, 0, 0x2000, 0x3000, None) == C.MLA_ERR_INVALID_ARG
+    assert L.mla_get_metadata(0x1000, 2, 1, 16, 1, 100, 8, 0x2000, 0x3000, None) == C.MLA_ERR_INVALID_ARG
+    assert L.mla_get_metadata(None, 2, 1, 16, 1, 0, 8, 0x2000, 0x3000, None) == C.MLA_ERR_INVALID_ARG
+    assert L.mla_get_metadata(0x1000, 2, 1, 16, 2, 0, 8, 0x2000, 0x3000, None) == C.MLA_ERR_UNSUPPORTED
+    assert L.mla_combine(None, 0, None, 1, 1, 1, None, None, None) == C.MLA_ERR_INVALID_ARG
+    assert L.mla_query_device_status(None, None, None) == C.MLA_ERR_INVALID_ARG
+
+
+def host_schedule(seqlens, batch, s_q, h_q, topk, parts):
+    U = batch * s_q if topk else batch
+    md = np.zeros(parts * 8, dtype=np.int32)
+    ns = np.zeros(U + 1, dtype=np.int32)
+    sl = np.ascontiguousarray(np.asarray(seqlens, dtype=np.int32))
+    assert M.mla_get_metadata_host(sl, batch, s_q, h_q, 1, topk, parts, md, ns) == 0
+    return md, ns
+
+
+@pytest.mark.parametrize("case", [
+    ("tiny", [70, 129], 1, 16, 0, 148),
+    ("dsv3", [4096] * 64, 1, 128, 0, 74),
+    ("single", [65536], 2, 16, 0, 148),
+    ("zeros", [0, 5, 0, 0, 300, 0], 1, 16, 0, 7),
+    ("all_zero", [0, 0, 0], 1, 16, 0, 5),
+    ("more_parts_than_tiles", [1, 2, 3], 1, 64, 0, 148),
+    ("sparse", [32768] * 32, 1, 128, 2048, 74),
+    ("sparse_sq2", [4096] * 3, 2, 64, 192, 11),
+])
+def test_host_scheduler_invariants(case):
+    _, lens, s_q, h_q, topk, parts = case
+    md, ns = host_schedule(lens, len(lens), s_q, h_q, topk, parts)
+    S.check_schedule(md, ns, lens, len(lens), s_q, topk, parts)
+
+
+def test_host_scheduler_random_and_mtp():
+    rng = np.random.default_rng(3)
+    for _ in range(40):
+        B = int(rng.integers(1, 300))
+        lens = rng.integers(0, 20000, size=B)
+        lens[rng.random(B) < 0.1] = 0
+        parts = int(rng.integers(1, 160))
+        md, ns = host_schedule(lens, B, 1, 16, 0, parts)
+        S.check_schedule(md, ns, lens, B, 1, 0, parts)
+    from workloads import mla_workloads as W
+    w = W.get_workload("mtp")
+    md, ns = host_schedule(w.seqlens, w.batch, 2, 16, 0, 148)
+    info = S.check_schedule(md, ns, w.seqlens, w.batch, 2, 0, 148)
+    assert info["splits"] <= w.batch + 148

@@ -1,0 +1,177 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle."""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import head_latent_attention_get_b200 as M
+from head_latent_attention_get_b200 import _capi as C
+from oracle import mla_oracle as O
+from tests import gpu_helpers as G
+from tests import sched_checks as S
+from workloads import mla_workloads as W
+
+pytestmark = pytest.mark.gpu
+
+
+def _dense(name="tiny", **over):
+    return dataclasses.replace(W.get_workload(name), **over)
+
+
+# ------------------------------------------------------------------ scheduler
+@pytest.mark.parametrize("lens,s_q,h_q,topk", [
+    ([70, 129], 1, 16, 0), ([4096] * 64, 1, 128, 0), ([0, 5, 0, 300, 9000], 2, 16, 0),
+    (list(range(0, 30000, 97)), 1, 64, 0), ([32768] * 32, 1, 128, 2048), ([100] * 5, 2, 32, 128)])
+def test_metadata_device_matches_host_twin(lens, s_q, h_q, topk):
+    B = len(lens)
+    parts = M.mla_get_num_sm_parts(0, s_q, h_q, 1, topk)
+    U = B * s_q if topk else B
+    md_h = np.zeros(parts * 8, np.int32)
+    ns_h = np.zeros(U + 1, np.int32)
+    lens_np = np.asarray(lens, np.int32)
+    assert M.mla_get_metadata_host(lens_np, B, s_q, h_q, 1, topk, parts, md_h, ns_h) == 0
+    md_d = torch.full((parts * 8,), -7, dtype=torch.int32, device="cuda")
+    ns_d = torch.full((U + 1,), -7, dtype=torch.int32, device="cuda")
+    M.mla_get_metadata(torch.from_numpy(lens_np).cuda(), B, s_q, h_q, 1, topk, parts, md_d, ns_d)
+    torch.cuda.synchronize()
+    assert np.array_equal(md_d.cpu().numpy(), md_h) and np.array_equal(ns_d.cpu().numpy(), ns_h)
+    S.check_schedule(md_h, ns_h, lens, B, s_q, topk, parts)
+
+
+# ------------------------------------------------------------------ combine
+def test_combine_matches_oracle_merge():
+    rng = np.random.default_rng(5)
+    U, R, parts = 3, 16, 4
+    n_splits = [3, 1, 0]            # unit 1 untouched (single split), unit 2 empty
+    ptr = np.concatenate([[0], np.cumsum(n_splits)]).astype(np.int32)
+    ws_bytes = M.mla_workspace_size(U, 1, R, 1, 0, parts)
+    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device="cuda")
+    q = rng.standard_normal((R, 576))
+    k = rng.standard_normal((300, 576))
+    cuts = [0, 64, 64, 300]           # the middle split has no keys
+    parts_o, parts_l = [], []
+    for a, b in zip(cuts[:-1], cuts[1:]):
+        o, l = O.attend(q, k[a:b], 1 / 24)
+        parts_o.append(o)
+        parts_l.append(l)
+    max_splits = U + parts
+    lse_off = 256
+    o_off = -(-(lse_off + max_splits * R * 4) // 256) * 256
+    lse_buf = np.zeros((max_splits, R), np.float32)
+    o_buf = np.zeros((max_splits, R, 512), np.float32)
+    for s in range(3):
+        lse_buf[s] = parts_l[s]
+        o_buf[s] = parts_o[s]
+    ws[lse_off:lse_off + lse_buf.nbytes] = torch.from_numpy(lse_buf.view(np.uint8).ravel()).cuda()
+    ws[o_off:o_off + o_buf.nbytes] = torch.from_numpy(o_buf.view(np.uint8).ravel()).cuda()
+    out = torch.full((U * R, 512), 7.0, dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((U * R,), 7.0, dtype=torch.float32, device="cuda")
+    M.mla_combine(ws, ws_bytes, torch.from_numpy(ptr).cuda(), U, R, parts, out, lse)
+    torch.cuda.synchronize()
+    ref_o, ref_l = O.combine(np.stack(parts_o), np.stack(parts_l))
+    G.compare(out[:R].float().cpu().numpy(), lse[:R].cpu().numpy(), ref_o, ref_l, "combine")
+    assert torch.all(out[R:2 * R] == 7.0) and torch.all(lse[R:2 * R] == 7.0)      # single split: untouched
+    assert torch.all(out[2 * R:] == 0) and torch.all(torch.isneginf(lse[2 * R:]))  # empty unit
+
+
+# ------------------------------------------------------------------ dense bf16
+def test_tiny_workload_full():
+    inp = W.make_inputs(W.get_workload("tiny"), poison_tail=True, extra_pages=2)
+    out, lse, _ = G.run_gpu(inp)
+    ref_o, ref_l = G.oracle_for(inp)
+    G.compare(out, lse, ref_o, ref_l, "tiny")
+
+
+@pytest.mark.parametrize("lens,s_q,h_q,causal", [
+    ([1, 63, 64, 65], 1, 16, False),
+    ([127, 128, 129, 255, 256, 257], 1, 32, False),
+    ([300, 1000, 2049], 1, 64, False),
+    ([700, 1500], 1, 128, False),
+    ([1, 2, 65, 129, 4000], 2, 16, True),
+    ([5, 300], 2, 32, True),
+    ([0, 100, 0], 1, 16, False),
+    ([3000], 2, 64, True),
+])
+def test_dense_shapes_vs_oracle(lens, s_q, h_q, causal):
+    w = _dense(batch=len(lens), seqlens=lens, s_q=s_q, h_q=h_q, causal=causal, seed=11 + sum(lens))
+    inp = W.make_inputs(w, poison_tail=True, extra_pages=3)
+    out, lse, r = G.run_gpu(inp)
+    ref_o, ref_l = G.oracle_for(inp)
+    G.compare(out, lse, ref_o, ref_l, f"{lens} s_q={s_q} h_q={h_q}")
+    assert r.status()[0] == C.MLA_OK
+
+
+@pytest.mark.parametrize("parts", [1, 2, 7, 148])
+def test_split_counts_do_not_change_results(parts):
+    w = _dense(batch=3, seqlens=[900, 4000, 130], h_q=64, seed=77)
+    inp = W.make_inputs(w, poison_tail=True)
+    out, lse, _ = G.run_gpu(inp, runner_kwargs={"num_sm_parts": parts})
+    ref_o, ref_l = G.oracle_for(inp)
+    G.compare(out, lse, ref_o, ref_l, f"parts={parts}")
+
+
+def test_dsv3_full_size_sampled():
+    inp = W.make_inputs(W.get_workload("dsv3"))
+    out, lse, _ = G.run_gpu(inp)
+    req = [0, 17, 63]
+    sub = G.restrict(inp, req)
+    ref_o, ref_l = G.oracle_for(sub)
+    G.compare(out[req], lse[req], ref_o, ref_l, "dsv3 sampled")
+    assert np.isfinite(lse).all() and np.isfinite(out).all()
+
+
+def test_mtp_full_size_sampled():
+    inp = W.make_inputs(W.get_workload("mtp"))
+    out, lse, _ = G.run_gpu(inp)
+    req = [0, 1, 127]
+    sub = G.restrict(inp, req)
+    ref_o, ref_l = G.oracle_for(sub)
+    G.compare(out[req], lse[req], ref_o, ref_l, "mtp sampled")
+    assert np.isfinite(lse).all()
+
+
+# ------------------------------------------------------------------ fp8 cache
+@pytest.mark.parametrize("lens,h_q", [([70, 129], 16), ([1, 64, 300], 64), ([1000, 2000], 128)])
+def test_fp8_vs_oracle_on_dequantised_values(lens, h_q):
+    w = _dense("fp8", batch=len(lens), seqlens=lens, h_q=h_q, seed=31 + sum(lens))
+    inp = W.make_inputs(w, poison_tail=True, extra_pages=1)
+    out, lse, _ = G.run_gpu(inp)
+    ref_o, ref_l = G.oracle_for(inp)
+    G.compare(out, lse, ref_o, ref_l, f"fp8 {lens}")
+
+
+def test_fp8_full_size_sampled():
+    inp = W.make_inputs(W.get_workload("fp8"))
+    out, lse, _ = G.run_gpu(inp)
+    req = [0, 40]
+    sub = G.restrict(inp, req)
+    ref_o, ref_l = G.oracle_for(sub)
+    G.compare(out[req], lse[req], ref_o, ref_l, "fp8 sampled")
+
+
+# ------------------------------------------------------------------ device status
+def test_bounds_status_without_fault():
+    w = _dense(batch=2, seqlens=[130, 64])
+    inp = W.make_inputs(w)
+    inp.block_table[0, 1] = inp.num_pages + 5          # out-of-range page id
+    out, lse, r = G.run_gpu(inp)
+    code, bits = r.status()
+    assert code == C.MLA_ERR_DEVICE_BOUNDS and bits & C.MLA_DEVICE_STATUS_BOUNDS
+    # the request that is in range is still exact
+    sub = G.restrict(inp, [1])
+    ref_o, ref_l = G.oracle_for(sub)
+    G.compare(out[1:], lse[1:], ref_o, ref_l, "unaffected request")
+
+
+def test_timeout_status_and_context_survives():
+    inp = W.make_inputs(W.get_workload("tiny"))
+    _, _, r = G.run_gpu(inp, runner_kwargs={"timeout_ns": 20_000_000,
+                                            "debug_flags": C.MLA_DEBUG_WITHHOLD_SCORES})
+    code, bits = r.status()
+    assert code == C.MLA_ERR_DEVICE_TIMEOUT and bits & C.MLA_DEVICE_STATUS_TIMEOUT
+    # the context is still usable: a normal call succeeds afterwards
+    out, lse, r2 = G.run_gpu(inp)
+    ref_o, ref_l = G.oracle_for(inp)
+    G.compare(out, lse, ref_o, ref_l, "after timeout")
+    assert r2.status()[0] == C.MLA_OK

@@ -248,3 +248,27 @@ def algorithmic_work(inp: DecodeInputs) -> dict:
         byts += sum((L + PAGE - 1) // PAGE for L in seqlens) * 4       # block-table entries read
     byts += w.batch * 4                                               # cache_seqlens
     return {"flops": flops, "bytes": float(byts), "keys": keys, "tokens_touched": touched}
+
+
+def restrict(inp: DecodeInputs, requests) -> DecodeInputs:
+    """Sub-problem with only the given requests and only their pages (block
+    table remapped). Each request's key set and values are unchanged, so a
+    sampled check or a bounded CPU-baseline sample can run on it without
+    touching the whole cache."""
+    import dataclasses
+    requests = list(requests)
+    bt = inp.block_table.numpy()
+    lens = inp.cache_seqlens.numpy()
+    pages = []
+    new_bt = np.full((len(requests), bt.shape[1]), -1, dtype=np.int32)
+    for i, b in enumerate(requests):
+        n = (int(lens[b]) + PAGE - 1) // PAGE
+        for j in range(n):
+            new_bt[i, j] = len(pages)
+            pages.append(int(bt[b, j]))
+    sub_lens = [int(lens[b]) for b in requests]
+    w = dataclasses.replace(inp.workload, batch=len(requests), seqlens=sub_lens)
+    return DecodeInputs(
+        workload=w, q=inp.q[requests].clone(), kcache=inp.kcache[pages].clone(),
+        block_table=torch.from_numpy(new_bt), cache_seqlens=torch.tensor(sub_lens, dtype=torch.int32),
+        indices=None if inp.indices is None else inp.indices[requests].clone())
