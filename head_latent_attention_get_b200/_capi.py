@@ -31,6 +31,7 @@ MLA_DEBUG_WITHHOLD_SCORES = 1
 MLA_DEBUG_SKIP_COMBINE = 2
 MLA_TILE_MD_INTS = 8
 MLA_MAX_ROWS = 128
+MLA_NOALLOC_WORKSPACE_BYTES = 48 << 20
 
 
 class MLAError(RuntimeError):
@@ -76,6 +77,8 @@ def lib() -> ctypes.CDLL:
         L.mla_workspace_size.argtypes = [i, i, i, i, i, i]
         L.mla_decode_paged.restype = i
         L.mla_decode_paged.argtypes = [ctypes.POINTER(MlaDecodeArgs), vp]
+        L.mla_decode_paged_noalloc.restype = i
+        L.mla_decode_paged_noalloc.argtypes = [ctypes.POINTER(MlaDecodeArgs), vp]
         L.mla_decode_sparse.restype = i
         L.mla_decode_sparse.argtypes = [ctypes.POINTER(MlaDecodeArgs), vp, i, vp]
         L.mla_combine.restype = i
@@ -160,6 +163,13 @@ def make_args(*, q, kcache, block_table, cache_seqlens, tile_md, num_splits, out
 
 def mla_decode_paged(args: MlaDecodeArgs, stream=None):
     _check(lib().mla_decode_paged(ctypes.byref(args), _stream(stream)), "mla_decode_paged")
+
+
+def mla_decode_paged_noalloc(args: MlaDecodeArgs, stream=None):
+    """Paged decode using the library's built-in workspace (args.workspace must
+    be None and args.workspace_bytes 0). For callers that cannot allocate
+    device memory at decode time."""
+    _check(lib().mla_decode_paged_noalloc(ctypes.byref(args), _stream(stream)), "mla_decode_paged_noalloc")
 
 
 def mla_decode_sparse(args: MlaDecodeArgs, indices, topk: int, stream=None):

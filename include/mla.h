@@ -187,6 +187,31 @@ typedef struct {
  * MLA_MAX_ROWS), WORKSPACE_TOO_SMALL, CUDA (launch failure). */
 mla_status_t mla_decode_paged(const mla_decode_args* args, mla_stream_t stream);
 
+/* Paged decoding with a built-in workspace (the pages have no counterpart:
+ * this entry point exists for callers that cannot allocate device memory
+ * when they decode, such as a server that reserved all device memory for its
+ * own pool at start-up, or a latency-critical step that must not pay for the
+ * implicit synchronisation and latency of cudaMalloc/cudaFree).
+ *
+ * Same computation and arguments as mla_decode_paged, except that
+ * args->workspace must be NULL and args->workspace_bytes 0: the split-KV
+ * partials and the device status word live in a file-scope device array of
+ * MLA_NOALLOC_WORKSPACE_BYTES held by every GPU that loads the library until
+ * the process exits. Nothing is allocated by the call.
+ *   - The first call on a device looks up the array's device address (once
+ *     per device, with that device current); make that first call before any
+ *     stream capture.
+ *   - All calls on a device share the array and it keeps the last call's
+ *     contents; calls whose work overlaps on the GPU race on it.
+ *   - Each call zeroes the status word before enqueueing the decode; device
+ *     status bits are not reported through mla_query_device_status (the
+ *     caller has no workspace pointer to pass).
+ * Errors: as mla_decode_paged; INVALID_ARG when a workspace is passed;
+ * WORKSPACE_TOO_SMALL when mla_workspace_size(...) of the problem exceeds
+ * MLA_NOALLOC_WORKSPACE_BYTES (use fewer num_sm_parts or mla_decode_paged). */
+#define MLA_NOALLOC_WORKSPACE_BYTES (48u << 20)
+mla_status_t mla_decode_paged_noalloc(const mla_decode_args* args, mla_stream_t stream);
+
 /* Token-sparse decoding. indices: device int32 [batch, s_q, topk], logical
  * token positions of request b resolved through its block-table row; -1
  * entries are ignored; other values outside [0, cache_seqlens[b]) are ignored
