@@ -76,19 +76,16 @@ mla_status_t check_common(const mla_decode_args* a, int topk) {
 mla_status_t run_decode(const mla_decode_args* a, const int32_t* indices, int topk, cudaStream_t stream) {
   const int rows = rows_of(a->s_q, a->h_q, a->h_kv, topk);
   const int U = units_of(a->batch, a->s_q, topk);
-  const int mode = topk > 0 ? 2 : (a->kv_format == MLA_KV_FP8_E4M3 ? 1 : 0);
-  CUtensorMap tq, tkv, taux;
+  const int mode = topk > 0 ? kModeSparse : (a->kv_format == MLA_KV_FP8_E4M3 ? kModeFp8 : kModeBf16);
+  // Q rows of every unit, and (bf16 paged cache only) the cache as
+  // [pages*64 tokens][576 dims]; boxes of 64 x 64 with 128-B swizzle. The FP8
+  // and sparse modes read the cache with cp.async and need no cache map.
+  CUtensorMap tq, tkv;
   std::memset(&tkv, 0, sizeof(tkv));
-  std::memset(&taux, 0, sizeof(taux));
   if (!make_map(&tq, a->q, (uint64_t)U * rows, kDqk, kDqk * 2, 64, 64)) return MLA_ERR_CUDA;
-  const uint64_t cache_rows = (uint64_t)a->num_pages * kPage;
-  if (mode == 1) {
-    // the 64 RoPE dims of each 656-byte record, read as bf16 columns 264..327
-    if (!make_map(&taux, a->kcache, cache_rows, kFp8RecordBytes / 2, kFp8RecordBytes, 64, 64)) return MLA_ERR_CUDA;
-  } else {
-    if (!make_map(&tkv, a->kcache, cache_rows, kDqk, kDqk * 2, 64, 64)) return MLA_ERR_CUDA;
-    if (mode == 2 && !make_map(&taux, a->kcache, cache_rows, kDqk, kDqk * 2, 64, 1)) return MLA_ERR_CUDA;
-  }
+  if (mode == kModeBf16 &&
+      !make_map(&tkv, a->kcache, (uint64_t)a->num_pages * kPage, kDqk, kDqk * 2, 64, 64))
+    return MLA_ERR_CUDA;
   const WsLayout w = ws_layout(U, rows, a->num_sm_parts);
   char* ws = static_cast<char*>(a->workspace);
   DecodeParams p;
@@ -107,6 +104,7 @@ mla_status_t run_decode(const mla_decode_args* a, const int32_t* indices, int to
   p.seqlens = a->cache_seqlens;
   p.indices = indices;
   p.kcache_fp8 = static_cast<const uint8_t*>(a->kcache);
+  p.kcache = a->kcache;
   p.tile_md = a->tile_md;
   p.split_ptr = a->num_splits;
   p.out = a->out;
@@ -118,7 +116,7 @@ mla_status_t run_decode(const mla_decode_args* a, const int32_t* indices, int to
   p.debug_flags = a->debug_flags;
   const int row_groups = (rows + kRowsPerCta - 1) / kRowsPerCta;
   const int rows_per_cta = rows < kRowsPerCta ? rows : kRowsPerCta;
-  if (launch_decode(rows_per_cta, mode, tq, tkv, taux, p, a->num_sm_parts, row_groups, stream) != cudaSuccess)
+  if (launch_decode(rows_per_cta, mode, tq, tkv, p, a->num_sm_parts, row_groups, stream) != cudaSuccess)
     return MLA_ERR_CUDA;
   if (a->debug_flags & MLA_DEBUG_SKIP_COMBINE) return MLA_OK;
   return launch_combine(a->workspace, U, rows, a->num_sm_parts, a->num_splits, a->out, a->lse, stream);

@@ -13,20 +13,26 @@
 //   softmax      one thread per query row reads its 128 scores from TMEM;
 //                online max / sum in fp32 with lazily rescaled O.
 //   O^T += V^T P^T  tcgen05 M=128 (4 chunks of the 512 value dims) x N=rows x
-//                K=128 tokens; V^T is the MN-major view of the token-major V
-//                tile, P^T (bf16) is written K-major by the row threads.
+//                K=64 tokens per V slot; V^T is the MN-major view of the
+//                token-major V tile, P^T (bf16) is written K-major by the row
+//                threads.
 // The O accumulator is transposed (value dims on TMEM lanes) so 64 rows x 512
 // dims fit in 256 TMEM columns next to two S buffers (2 x 128 columns).
-// K slices and V chunks stream through separate smem rings (V is read again
-// from L2 for the PV product) so the ring stays several slots deep.
+// K slices (128 tokens x 64 dims) and V slots (64 tokens x 128 dims) stream
+// through separate 4-slot smem rings; V is read a second time (from L2) for
+// the PV product rather than held across the softmax, which keeps the rings
+// deep enough to cover the load latency.
 //
-// Warp roles (256 threads; 384 with the FP8 cache):
-//   0 K producer (Q + K slices via TMA)     1 S issuer (+ TMEM alloc)
-//   2 O issuer                              3 V producer (V chunks via TMA)
+// Warp roles (256 threads; 320 with the FP8 cache or sparse indices):
+//   0 Q (and, bf16 paged, K slices) via TMA   1 S issuer (+ TMEM alloc)
+//   2 O issuer                                 3 V slots via TMA (bf16 paged)
 //   4-7 softmax + epilogue (row r = 16*(warp-4) + lane, lanes 0-15)
-//   8-9 FP8 dequant of K slices 0-7         10-11 FP8 dequant of V chunks
+//   8 K gather warp, 9 V gather warp (FP8 / sparse): cp.async copies
+//       software-pipelined three slots deep; FP8 codes are converted in place.
 // Every mbarrier wait is bounded; on timeout the CTA records
-// MLA_DEVICE_STATUS_TIMEOUT, stops issuing work and exits normally.
+// MLA_DEVICE_STATUS_TIMEOUT, stops issuing work, waits (bounded) for its own
+// copies in flight and exits normally. Every ring has exactly one producer
+// role so that no parity wait can fall two phases behind.
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
@@ -36,23 +42,25 @@
 
 namespace mla {
 
-constexpr int kNK = 3;                 // K ring slots (16 KB: 128 tokens x 64 dims)
-constexpr int kNV = 2;                 // V ring slots (32 KB: 128 tokens x 128 dims)
+constexpr int kNK = 4;                 // K ring slots: 128 tokens x 64 dims (16 KB)
+constexpr int kNV = 4;                 // V ring slots: 64 tokens x 128 dims (16 KB)
+constexpr int kSlot = 16384;
+constexpr int kLag = 3;                // gather groups retire a slot 3 slots after issuing it
+constexpr int kPrefetchTiles = 3;      // L2 prefetch distance (bf16 paged)
 constexpr int kQBytes = 9 * 8192;      // 64 rows x 576 dims
-constexpr int kKSlot = 16384;
-constexpr int kVSlot = 32768;
 constexpr int kTmemCols = 512;
 constexpr int kTmemS = 256;            // S buffers at columns 256 and 384
 constexpr float kRescaleLog2 = 8.0f;   // rescale O only when the max grows by > 2^8
+static_assert(kLag < kNK && kLag < kNV, "a gather group must retire a slot before reusing it");
 
 template <int NR>
 struct Smem {
   static constexpr int q = 0;
   static constexpr int k = q + kQBytes;
-  static constexpr int v = k + kNK * kKSlot;
-  static constexpr int pt = v + kNV * kVSlot;
+  static constexpr int v = k + kNK * kSlot;
+  static constexpr int pt = v + kNV * kSlot;
   static constexpr int pt_bytes = NR * 256;  // [NR rows][128 tokens] bf16
-  static constexpr int ctrl = pt + 2 * pt_bytes;
+  static constexpr int ctrl = pt + pt_bytes;
   static constexpr int total = ctrl + 1024;
 };
 
@@ -60,8 +68,9 @@ struct Ctrl {
   uint64_t q_full, q_empty;
   uint64_t k_full[kNK], k_empty[kNK];
   uint64_t v_full[kNV], v_empty[kNV];
-  uint64_t s_full[2], s_empty[2], p_full[2], o_done[2], o_free, drain_s, drain_o;
-  uint64_t grp_sm, grp_k, grp_v;   // bounded group barriers (softmax 128, dequant 64 + 64)
+  uint64_t s_full[2], s_empty[2];
+  uint64_t p_full, o_done, o_free, drain_s, drain_o;
+  uint64_t grp_sm;  // bounded barrier of the 128 softmax threads
   uint32_t tmem_base;
   int abort_flag;
   int rescale_flag[2];
@@ -132,15 +141,15 @@ __device__ __forceinline__ bool group_sync(Ctrl* c, uint64_t* bar, uint32_t& pha
   return ok;
 }
 
-// Before a producer exits (normally or after an abort) it waits, with a bound,
-// for the copies it issued into its last `nslots` ring slots, so no TMA write
-// can land in shared memory after the CTA has finished.
+// Before a TMA producer exits (normally or after an abort) it waits, with a
+// bound, for the copies it issued into its last `nslots` ring slots, so no TMA
+// write can land in shared memory after the CTA has finished.
 __device__ __forceinline__ void drain_issued(uint64_t* full, int nslots, int issued, uint64_t timeout_ns) {
   for (int i = issued > nslots ? issued - nslots : 0; i < issued; ++i)
     mbar_wait(&full[i % nslots], (uint32_t)((i / nslots) & 1), timeout_ns);
 }
 
-// Physical page of logical page j of unit u (dense); -1 when j is past the
+// Physical page of logical page j of a request (dense); -1 when j is past the
 // request's pages. Out-of-range ids are reported and replaced by page 0.
 __device__ __forceinline__ int page_of(const DecodeParams& p, int req, int j, int npages_req) {
   if (j >= npages_req) return -1;
@@ -206,15 +215,173 @@ __device__ __forceinline__ void dequant16(const uint4 raw, float s, uint4& lo, u
   hi = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
-// Store 16 bytes at chunk c (0..7) of 128-B row `row` of a 128-B-swizzled tile.
-__device__ __forceinline__ void st_sw128(uint8_t* tile, int row, int c, uint4 v) {
-  *reinterpret_cast<uint4*>(tile + row * 128 + ((c ^ (row & 7)) << 4)) = v;
+// Address of 16-byte chunk c (0..7) of 128-B row `row` of a 128-B-swizzled tile.
+__device__ __forceinline__ uint8_t* sw128(uint8_t* tile, int row, int c) {
+  return tile + row * 128 + ((c ^ (row & 7)) << 4);
 }
 
+__device__ __forceinline__ float pick4(const float4 v, int i) {
+  return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
+__device__ __forceinline__ uint32_t pick4u(const uint4 v, int i) {
+  return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
+
+// ============================================================================ gather groups
+// FP8 and sparse modes: one warp fills the K ring and one warp the V ring with
+// 16-byte cp.async copies. Each lane issues the copies of a slot, commits them
+// as one group and retires the slot it issued kLag slots earlier: wait for
+// that group, convert it (FP8), fence the generic-proxy writes for the tensor
+// core, arrive on the slot's full barrier (count 32).
+// Lane t copies tokens t + 32q of a 128-token tile (q = 0..3); a V slot holds
+// the 64 tokens of one page, so lane t copies its tokens t and t + 32 there.
+constexpr int kGatherLanes = 32;
+
+struct GatherRing {
+  uint64_t* full;
+  uint64_t* empty;
+  uint8_t* base;
+  int nslots;
+};
+
+template <int MODE, bool KGROUP>
+__device__ __forceinline__ void retire_slot(const GatherRing& g, int seq, int t) {
+  const int slot = seq % g.nslots;
+  uint8_t* s = g.base + slot * kSlot;
+  if (MODE == kModeFp8) {
+    if (KGROUP) {
+      const int j = seq % 9;
+      if (j != 8) {  // latent slice: codes in bytes [0,64) and scales in [64,80) of the row
+#pragma unroll 1
+        for (int q = 0; q < 4; ++q) {
+          const int row = t + 32 * q;
+          const uint4* raw = reinterpret_cast<const uint4*>(s + row * 128);
+          uint4 cw[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) cw[i] = raw[i];
+          const float scale = pick4(*reinterpret_cast<const float4*>(s + row * 128 + 64), j >> 1);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            uint4 lo, hi;
+            dequant16(cw[i], scale, lo, hi);
+            *reinterpret_cast<uint4*>(sw128(s, row, 2 * i)) = lo;
+            *reinterpret_cast<uint4*>(sw128(s, row, 2 * i + 1)) = hi;
+          }
+        }
+      }
+    } else {  // V slot: codes in half-0 row, scales at the start of the half-1 row
+      const int m = (seq >> 1) & 3;
+#pragma unroll 1
+      for (int q = 0; q < 2; ++q) {
+        const int row = t + 32 * q;
+        const uint4* raw = reinterpret_cast<const uint4*>(s + row * 128);
+        uint4 cw[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) cw[i] = raw[i];
+        const float scale = pick4(*reinterpret_cast<const float4*>(s + 8192 + row * 128), m);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          uint4 lo, hi;
+          dequant16(cw[i], scale, lo, hi);
+          uint8_t* half = s + (i >> 2) * 8192;
+          *reinterpret_cast<uint4*>(sw128(half, row, 2 * (i & 3))) = lo;
+          *reinterpret_cast<uint4*>(sw128(half, row, 2 * (i & 3) + 1)) = hi;
+        }
+      }
+    }
+  }
+  fence_proxy_async_smem();
+  mbar_arrive(&g.full[slot]);
+}
+
+template <int MODE, bool KGROUP>
+__device__ void gather_group(const DecodeParams& p, Ctrl* c, PieceIter& it, const GatherRing& g, int t) {
+  int seq = 0;       // slots issued
+  int retired = 0;   // slots retired
+  bool stop = false;
+  Piece pc;
+  while (!stop && it.next(pc)) {
+    const int unit = pc.unit;
+    const int req = unit_req(p, unit);
+    const int npg = (MODE == kModeSparse) ? 0 : (p.seqlens[req] + kPage - 1) / kPage;
+    for (int k = pc.t0; k < pc.t1 && !stop; ++k) {
+      // source rows of tokens t + 32q of the tile (q = 0..3)
+      const uint8_t* src[4];
+      uint32_t ok[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int tt = t + 32 * q;
+        if (MODE == kModeSparse) {
+          const int row = sparse_row(p, unit, k * kTile + tt, KGROUP);
+          ok[q] = row >= 0 ? 16u : 0u;  // ignored slots are zero-filled
+          src[q] = static_cast<const uint8_t*>(p.kcache) + (size_t)(row >= 0 ? row : 0) * (kDqk * 2);
+        } else {
+          int pg = page_of(p, req, 2 * k + (tt >> 6), npg);
+          if (pg < 0) pg = page_of(p, req, 2 * k, npg);
+          ok[q] = 16u;
+          src[q] = p.kcache_fp8 + ((size_t)pg * kPage + (tt & 63)) * kFp8RecordBytes;
+        }
+      }
+      const int slots_per_tile = KGROUP ? 9 : 8;
+      for (int j = 0; j < slots_per_tile; ++j, ++seq) {
+        const int slot = seq % g.nslots;
+        uint8_t* s = g.base + slot * kSlot;
+        if (!timed_wait(c, &g.empty[slot], ((seq / g.nslots) & 1) ^ 1, p)) { stop = true; break; }
+        if (KGROUP) {  // slice j (64 dims) of the four tokens
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int row = t + 32 * q;
+            if (MODE == kModeSparse) {
+#pragma unroll
+              for (int ch = 0; ch < 8; ++ch) cp_async16(sw128(s, row, ch), src[q] + 128 * j + 16 * ch, ok[q]);
+            } else if (j == 8) {  // RoPE dims: bf16 straight into place
+#pragma unroll
+              for (int ch = 0; ch < 8; ++ch) cp_async16(sw128(s, row, ch), src[q] + 528 + 16 * ch, 16u);
+            } else {  // latent codes + scales into the row, converted at retire
+#pragma unroll
+              for (int ch = 0; ch < 4; ++ch) cp_async16(s + row * 128 + 16 * ch, src[q] + 64 * j + 16 * ch, 16u);
+              cp_async16(s + row * 128 + 64, src[q] + 512, 16u);
+            }
+          }
+        } else {  // V slot j: value dims 128*(j/2).., page half h = j%2, tokens t and t+32 of it
+          const int m = j >> 1, h = j & 1;
+#pragma unroll
+          for (int qq = 0; qq < 2; ++qq) {
+            const int q = 2 * h + qq, row = t + 32 * qq;
+            if (MODE == kModeSparse) {
+#pragma unroll
+              for (int ch = 0; ch < 16; ++ch)
+                cp_async16(sw128(s + (ch >> 3) * 8192, row, ch & 7), src[q] + 256 * m + 16 * ch, ok[q]);
+            } else {
+#pragma unroll
+              for (int ch = 0; ch < 8; ++ch) cp_async16(s + row * 128 + 16 * ch, src[q] + 128 * m + 16 * ch, 16u);
+              cp_async16(s + 8192 + row * 128, src[q] + 512, 16u);
+            }
+          }
+        }
+        cp_async_commit();
+        if (seq + 1 - retired > kLag) {
+          cp_async_wait<kLag>();
+          retire_slot<MODE, KGROUP>(g, retired, t);
+          ++retired;
+        }
+      }
+    }
+  }
+  cp_async_wait<0>();  // no copy may land after the CTA has finished
+  if (!stop) {
+    while (retired < seq) {
+      retire_slot<MODE, KGROUP>(g, retired, t);
+      ++retired;
+    }
+  }
+}
+
+// ============================================================================ kernel
 template <int NR, int MODE>
-__global__ void __launch_bounds__(MODE == kModeFp8 ? 384 : 256, 1)
+__global__ void __launch_bounds__(MODE == kModeBf16 ? 256 : 320, 1)
     mla_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
-                      const __grid_constant__ CUtensorMap tm_aux, const DecodeParams p) {
+                      const DecodeParams p) {
   using L = Smem<NR>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -228,24 +395,20 @@ __global__ void __launch_bounds__(MODE == kModeFp8 ? 384 : 256, 1)
   const int part = blockIdx.x, rg = blockIdx.y;
   const int row0 = rg * kRowsPerCta;                    // first row of this CTA within a unit
   const int rows_here = min(kRowsPerCta, p.rows - row0);
+  constexpr uint32_t kFullCount = MODE == kModeBf16 ? 1 : kGatherLanes;
 
   if (threadIdx.x == 0) {
     mbar_init(&c->q_full, 1);
     mbar_init(&c->q_empty, 1);
-    for (int i = 0; i < kNK; ++i) { mbar_init(&c->k_full[i], 1); mbar_init(&c->k_empty[i], 1); }
-    for (int i = 0; i < kNV; ++i) { mbar_init(&c->v_full[i], 1); mbar_init(&c->v_empty[i], 1); }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&c->s_full[i], 1);
-      mbar_init(&c->s_empty[i], 128);
-      mbar_init(&c->p_full[i], 128);
-      mbar_init(&c->o_done[i], 1);
-    }
+    for (int i = 0; i < kNK; ++i) { mbar_init(&c->k_full[i], kFullCount); mbar_init(&c->k_empty[i], 1); }
+    for (int i = 0; i < kNV; ++i) { mbar_init(&c->v_full[i], kFullCount); mbar_init(&c->v_empty[i], 1); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&c->s_full[i], 1); mbar_init(&c->s_empty[i], 128); }
+    mbar_init(&c->p_full, 128);
+    mbar_init(&c->o_done, 1);
     mbar_init(&c->o_free, 128);
     mbar_init(&c->drain_s, 1);
     mbar_init(&c->drain_o, 1);
     mbar_init(&c->grp_sm, 128);
-    mbar_init(&c->grp_k, 64);
-    mbar_init(&c->grp_v, 64);
     c->abort_flag = 0;
     c->rescale_flag[0] = 0;
     c->rescale_flag[1] = 0;
@@ -253,8 +416,7 @@ __global__ void __launch_bounds__(MODE == kModeFp8 ? 384 : 256, 1)
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tm_q);
-    if (MODE == kModeBf16) tma_prefetch_desc(&tm_kv);  // the other map is left unencoded
-    else tma_prefetch_desc(&tm_aux);
+    if (MODE == kModeBf16) tma_prefetch_desc(&tm_kv);  // encoded only for the bf16 paged cache
   }
   if (warp == 1) {
     tmem_alloc(&c->tmem_base, kTmemCols);
@@ -270,7 +432,7 @@ __global__ void __launch_bounds__(MODE == kModeFp8 ? 384 : 256, 1)
   Piece pc;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ K producer
+    // ------------------------------------------------------------ Q (+ K slices, bf16)
     int kc = 0, pi = 0, q_issued = 0;
     bool stop = false;
     while (!stop && it.next(pc)) {
@@ -283,189 +445,76 @@ __global__ void __launch_bounds__(MODE == kModeFp8 ? 384 : 256, 1)
           for (int j = 0; j < 9; ++j) tma_load_2d(sQ + j * 8192, &tm_q, &c->q_full, 64 * j, qy);
           ++q_issued;
         }
+        if (MODE == kModeBf16 && !stop) {
+          const int req = pc.unit;
+          const int npg = (p.seqlens[req] + kPage - 1) / kPage;
+          for (int k = pc.t0; k < pc.t1 && !stop; ++k) {
+            int pa = page_of(p, req, 2 * k, npg);
+            int pb = page_of(p, req, 2 * k + 1, npg);
+            if (pb < 0) pb = pa;  // half tile: reload page A, its keys are masked
+            if (rg == 0 && k + kPrefetchTiles < pc.t1) {  // warm L2 a few tiles ahead
+              for (int h = 0; h < 2; ++h) {
+                const int pf = page_of(p, req, 2 * (k + kPrefetchTiles) + h, npg);
+                if (pf >= 0)
+                  prefetch_l2(static_cast<const uint8_t*>(p.kcache) + (size_t)pf * kPage * kDqk * 2,
+                              kPage * kDqk * 2);
+              }
+            }
+            for (int j = 0; j < 9; ++j, ++kc) {
+              const int slot = kc % kNK;
+              uint8_t* dst = sK + slot * kSlot;
+              if (!timed_wait(c, &c->k_empty[slot], ((kc / kNK) & 1) ^ 1, p)) { stop = true; break; }
+              mbar_arrive_expect_tx(&c->k_full[slot], kSlot);
+              tma_load_2d(dst, &tm_kv, &c->k_full[slot], 64 * j, pa * kPage);
+              tma_load_2d(dst + 8192, &tm_kv, &c->k_full[slot], 64 * j, pb * kPage);
+            }
+          }
+        }
       }
       stop = __shfl_sync(0xffffffffu, stop ? 1 : 0, 0) != 0;
-      if (stop) break;
-      const int req = unit_req(p, pc.unit);
-      const int npg = (MODE == kModeSparse) ? 0 : (p.seqlens[req] + kPage - 1) / kPage;
-      for (int k = pc.t0; k < pc.t1 && !stop; ++k) {
-        int pa = 0, pb = 0;
-        if (MODE != kModeSparse && lane == 0) {
-          pa = page_of(p, req, 2 * k, npg);
-          pb = page_of(p, req, 2 * k + 1, npg);
-          if (pb < 0) pb = pa;      // half tile: reload page A, its keys are masked
-        }
-        // sparse: lane l gathers slots 4l..4l+3 of this tile (ignored slots load
-        // row 0; their scores are masked and their value rows zeroed later)
-        int r4[4] = {0, 0, 0, 0};
-        if (MODE == kModeSparse) {
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int rr = sparse_row(p, pc.unit, k * kTile + 4 * lane + q, true);
-            r4[q] = rr < 0 ? 0 : rr;
-          }
-        }
-        if (MODE == kModeFp8) continue;  // the dequant group is the only producer of K slots
-        for (int j = 0; j < 9; ++j, ++kc) {
-          const int slot = kc % kNK;
-          uint8_t* dst = sK + slot * kKSlot;
-          if (lane == 0) {
-            if (!timed_wait(c, &c->k_empty[slot], ((kc / kNK) & 1) ^ 1, p)) { stop = true; }
-            else if (MODE == kModeSparse) mbar_arrive_expect_tx(&c->k_full[slot], kKSlot);
-          }
-          stop = __shfl_sync(0xffffffffu, stop ? 1 : 0, 0) != 0;
-          if (stop) break;
-          if (MODE == kModeSparse) {
-            __syncwarp();
-            tma_gather4(dst + lane * 512, &tm_aux, &c->k_full[slot], 64 * j, r4[0], r4[1], r4[2], r4[3]);
-          } else if (lane == 0) {
-            mbar_arrive_expect_tx(&c->k_full[slot], kKSlot);
-            tma_load_2d(dst, &tm_kv, &c->k_full[slot], 64 * j, pa * kPage);
-            tma_load_2d(dst + 8192, &tm_kv, &c->k_full[slot], 64 * j, pb * kPage);
-          }
-          __syncwarp();
-        }
-      }
       ++pi;
     }
     if (lane == 0) {
       if (q_issued > 0) mbar_wait(&c->q_full, (uint32_t)((q_issued - 1) & 1), p.timeout_ns);
-      if (MODE != kModeFp8) drain_issued(c->k_full, kNK, kc, p.timeout_ns);
+      if (MODE == kModeBf16) drain_issued(c->k_full, kNK, kc, p.timeout_ns);
     }
     __syncwarp();
-  } else if (warp == 3 && MODE != kModeFp8) {
-    // ------------------------------------------------------------ V producer
-    int vc = 0;
-    bool stop = false;
-    while (!stop && it.next(pc)) {
-      const int req = unit_req(p, pc.unit);
-      const int npg = (MODE == kModeSparse) ? 0 : (p.seqlens[req] + kPage - 1) / kPage;
-      for (int k = pc.t0; k < pc.t1 && !stop; ++k) {
-        int pa = 0, pb = 0;
-        if (MODE != kModeSparse && lane == 0) {
-          pa = page_of(p, req, 2 * k, npg);
-          pb = page_of(p, req, 2 * k + 1, npg);
-          if (pb < 0) pb = pa;
-        }
-        int r4[4];
-        if (MODE == kModeSparse) {
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int rr = sparse_row(p, pc.unit, k * kTile + 4 * lane + q, false);
-            r4[q] = rr < 0 ? 0 : rr;
-          }
-        }
-        for (int m = 0; m < 4; ++m, ++vc) {
-          const int slot = vc % kNV;
-          uint8_t* dst = sV + slot * kVSlot;
-          if (lane == 0) {
-            if (!timed_wait(c, &c->v_empty[slot], ((vc / kNV) & 1) ^ 1, p)) stop = true;
-            else mbar_arrive_expect_tx(&c->v_full[slot], kVSlot);
-          }
-          stop = __shfl_sync(0xffffffffu, stop ? 1 : 0, 0) != 0;
-          if (stop) break;
-          __syncwarp();
-          if (MODE == kModeSparse) {
-            tma_gather4(dst + lane * 512, &tm_aux, &c->v_full[slot], 128 * m, r4[0], r4[1], r4[2], r4[3]);
-            tma_gather4(dst + 16384 + lane * 512, &tm_aux, &c->v_full[slot], 128 * m + 64, r4[0], r4[1],
-                        r4[2], r4[3]);
-          } else if (lane == 0) {
-            tma_load_2d(dst, &tm_kv, &c->v_full[slot], 128 * m, pa * kPage);
-            tma_load_2d(dst + 8192, &tm_kv, &c->v_full[slot], 128 * m, pb * kPage);
-            tma_load_2d(dst + 16384, &tm_kv, &c->v_full[slot], 128 * m + 64, pa * kPage);
-            tma_load_2d(dst + 24576, &tm_kv, &c->v_full[slot], 128 * m + 64, pb * kPage);
-          }
-          __syncwarp();
-        }
-      }
-    }
-    if (lane == 0) drain_issued(c->v_full, kNV, vc, p.timeout_ns);
-    __syncwarp();
-  } else if (MODE == kModeFp8 && warp >= 8) {
-    // ------------------------------------------------------------ FP8 dequant
-    const bool kgroup = warp < 10;
-    const int gt = threadIdx.x - (kgroup ? 256 : 320);  // 0..63 within the group
-    uint64_t* grp = kgroup ? &c->grp_k : &c->grp_v;
-    uint32_t gph = 0;
-    int kc = 0, vc = 0;
-    bool stop = false;
-    while (!stop && it.next(pc)) {
-      const int req = pc.unit;
-      const int npg = (p.seqlens[req] + kPage - 1) / kPage;
-      for (int k = pc.t0; k < pc.t1 && !stop; ++k) {
-        // this thread converts tokens gt and gt + 64 of the tile
-        const uint8_t* rec[2];
-        int pgs[2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          int pg = page_of(p, req, 2 * k + h, npg);
-          if (pg < 0) pg = page_of(p, req, 2 * k, npg);
-          pgs[h] = pg;
-          rec[h] = p.kcache_fp8 + ((size_t)pg * kPage + gt) * kFp8RecordBytes;
-        }
-        if (kgroup) {
-          // this group is the only producer of the K ring (one producer keeps every
-          // empty-barrier wait at most one phase behind)
-          for (int j = 0; j < 9; ++j, ++kc) {
-            const int slot = kc % kNK;
-            uint8_t* dst = sK + slot * kKSlot;
-            if (j == 8) {  // RoPE slice straight from the records (bytes 528..655) by TMA
-              if (gt == 0) {
-                if (!timed_wait(c, &c->k_empty[slot], ((kc / kNK) & 1) ^ 1, p)) {
-                  stop = true;
-                } else {
-                  mbar_arrive_expect_tx(&c->k_full[slot], kKSlot);
-                  tma_load_2d(dst, &tm_aux, &c->k_full[slot], 264, pgs[0] * kPage);
-                  tma_load_2d(dst + 8192, &tm_aux, &c->k_full[slot], 264, pgs[1] * kPage);
-                }
-              }
-              continue;
-            }
-            if (gt == 0 && !timed_wait(c, &c->k_empty[slot], ((kc / kNK) & 1) ^ 1, p)) stop = true;
-            if (!group_sync(c, grp, gph, p) || *(volatile int*)&c->abort_flag) { stop = true; break; }
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const float s = reinterpret_cast<const float*>(rec[h] + 512)[j >> 1];
-              const uint4* src = reinterpret_cast<const uint4*>(rec[h] + 64 * j);
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                uint4 lo, hi;
-                dequant16(__ldg(src + q), s, lo, hi);
-                st_sw128(dst, gt + 64 * h, 2 * q, lo);
-                st_sw128(dst, gt + 64 * h, 2 * q + 1, hi);
-              }
-            }
-            fence_proxy_async_smem();
-            if (!group_sync(c, grp, gph, p)) { stop = true; break; }
-            if (gt == 0) mbar_arrive(&c->k_full[slot]);
-          }
-        } else {
-          for (int m = 0; m < 4; ++m, ++vc) {
+  } else if (warp == 3 && MODE == kModeBf16) {
+    // ------------------------------------------------------------ V slots (bf16)
+    if (lane == 0) {
+      int vc = 0;
+      bool stop = false;
+      while (!stop && it.next(pc)) {
+        const int req = pc.unit;
+        const int npg = (p.seqlens[req] + kPage - 1) / kPage;
+        for (int k = pc.t0; k < pc.t1 && !stop; ++k) {
+          int pg[2];
+          pg[0] = page_of(p, req, 2 * k, npg);
+          pg[1] = page_of(p, req, 2 * k + 1, npg);
+          if (pg[1] < 0) pg[1] = pg[0];
+          for (int j = 0; j < 8; ++j, ++vc) {  // slot j: value dims 128*(j/2).., page half j%2
             const int slot = vc % kNV;
-            uint8_t* dst = sV + slot * kVSlot;
-            if (gt == 0 && !timed_wait(c, &c->v_empty[slot], ((vc / kNV) & 1) ^ 1, p)) stop = true;
-            if (!group_sync(c, grp, gph, p) || *(volatile int*)&c->abort_flag) { stop = true; break; }
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const float s = reinterpret_cast<const float*>(rec[h] + 512)[m];
-              const uint4* src = reinterpret_cast<const uint4*>(rec[h] + 128 * m);
-#pragma unroll
-              for (int q = 0; q < 8; ++q) {
-                uint4 lo, hi;
-                dequant16(__ldg(src + q), s, lo, hi);
-                uint8_t* half = dst + (q >> 2) * 16384;   // dims 0-63 / 64-127 of the chunk
-                st_sw128(half, gt + 64 * h, 2 * (q & 3), lo);
-                st_sw128(half, gt + 64 * h, 2 * (q & 3) + 1, hi);
-              }
-            }
-            fence_proxy_async_smem();
-            if (!group_sync(c, grp, gph, p)) { stop = true; break; }
-            if (gt == 0) mbar_arrive(&c->v_full[slot]);
+            uint8_t* dst = sV + slot * kSlot;
+            if (!timed_wait(c, &c->v_empty[slot], ((vc / kNV) & 1) ^ 1, p)) { stop = true; break; }
+            mbar_arrive_expect_tx(&c->v_full[slot], kSlot);
+            const int m = j >> 1, y = pg[j & 1] * kPage;
+            tma_load_2d(dst, &tm_kv, &c->v_full[slot], 128 * m, y);
+            tma_load_2d(dst + 8192, &tm_kv, &c->v_full[slot], 128 * m + 64, y);
           }
         }
       }
+      drain_issued(c->v_full, kNV, vc, p.timeout_ns);
     }
-    if (kgroup && gt == 0) drain_issued(c->k_full, kNK, kc, p.timeout_ns);
+    __syncwarp();
+  } else if (MODE != kModeBf16 && warp >= 8) {
+    // ------------------------------------------------------------ gather groups
+    if (warp == 8) {
+      const GatherRing g{c->k_full, c->k_empty, sK, kNK};
+      gather_group<MODE, true>(p, c, it, g, lane);
+    } else {
+      const GatherRing g{c->v_full, c->v_empty, sV, kNV};
+      gather_group<MODE, false>(p, c, it, g, lane);
+    }
   } else if (warp == 1) {
     // ------------------------------------------------------------ S issuer
     const uint32_t idesc = idesc_bf16(64, 128, false, false);
@@ -483,7 +532,7 @@ __global__ void __launch_bounds__(MODE == kModeFp8 ? 384 : 256, 1)
             const int slot = kc % kNK;
             if (!timed_wait(c, &c->k_full[slot], (kc / kNK) & 1, p)) { stop = true; break; }
             tc_fence_after();
-            const uint32_t qa = smem_u32(sQ + j * 8192), kb = smem_u32(sK + slot * kKSlot);
+            const uint32_t qa = smem_u32(sQ + j * 8192), kb = smem_u32(sK + slot * kSlot);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
               mma_bf16_ss(d, sdesc(qa + kk * 32, 16, 1024), sdesc(kb + kk * 32, 16, 1024), idesc,
@@ -509,44 +558,30 @@ __global__ void __launch_bounds__(MODE == kModeFp8 ? 384 : 256, 1)
     while (!stop && it.next(pc)) {
       const int req = unit_req(p, pc.unit);
       for (int k = pc.t0; k < pc.t1 && !stop; ++k, ++gt) {
-        const int b = gt & 1;
         const bool first = (k == pc.t0);
         if (lane == 0) {
           if (first && pi > 0 && !timed_wait(c, &c->o_free, (pi - 1) & 1, p)) stop = true;
-          if (!stop && !timed_wait(c, &c->p_full[b], (gt >> 1) & 1, p)) stop = true;
+          if (!stop && !timed_wait(c, &c->p_full, gt & 1, p)) stop = true;
         }
         stop = __shfl_sync(0xffffffffu, stop ? 1 : 0, 0) != 0;
         if (stop) break;
-        // keys of this tile whose value rows must read as zero
-        int nvalid = kTile;
-        uint32_t bad = 0;  // sparse: bit i of lane l -> slot 4l + i ignored
-        if (MODE == kModeSparse) {
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            if (sparse_row(p, pc.unit, k * kTile + 4 * lane + q, false) < 0) bad |= 1u << q;
-        } else {
-          nvalid = dense_tile_valid(p.seqlens[req], k);
-        }
-        const uint32_t pt = smem_u32(sP + b * L::pt_bytes);
-        for (int m = 0; m < 4 && !stop; ++m, ++vc) {
+        // dense: value rows of keys past the request's end must read as zero
+        // (ignored sparse slots are zero-filled by the gather already)
+        const int nvalid = (MODE == kModeSparse) ? kTile : dense_tile_valid(p.seqlens[req], k);
+        const uint32_t pt = smem_u32(sP);
+        for (int j = 0; j < 8 && !stop; ++j, ++vc) {
           const int slot = vc % kNV;
-          uint8_t* vs = sV + slot * kVSlot;
+          const int m = j >> 1, h = j & 1;
+          uint8_t* vs = sV + slot * kSlot;
           if (lane == 0 && !timed_wait(c, &c->v_full[slot], (vc / kNV) & 1, p)) stop = true;
           stop = __shfl_sync(0xffffffffu, stop ? 1 : 0, 0) != 0;
           if (stop) break;
-          if (MODE == kModeSparse ? __any_sync(0xffffffffu, bad != 0) : nvalid < kTile) {
+          const int nv_slot = min(64, max(0, nvalid - 64 * h));
+          if (nv_slot < 64) {
             const uint4 z = make_uint4(0, 0, 0, 0);
-            if (MODE == kModeSparse) {
-              for (int q = 0; q < 4; ++q)
-                if (bad & (1u << q))
-                  for (int h = 0; h < 2; ++h)
-                    for (int ch = 0; ch < 8; ++ch)
-                      *reinterpret_cast<uint4*>(vs + h * 16384 + (4 * lane + q) * 128 + ch * 16) = z;
-            } else {
-              for (int i = nvalid * 16 + lane; i < kTile * 16; i += 32) {  // 16 chunks per token row
-                const int tok = i >> 4, ch = i & 15;
-                *reinterpret_cast<uint4*>(vs + (ch >> 3) * 16384 + tok * 128 + (ch & 7) * 16) = z;
-              }
+            for (int i = nv_slot * 16 + lane; i < 64 * 16; i += 32) {  // 16 chunks per token row
+              const int tok = i >> 4, ch = i & 15;
+              *reinterpret_cast<uint4*>(vs + (ch >> 3) * 8192 + tok * 128 + (ch & 7) * 16) = z;
             }
             fence_proxy_async_smem();
             __syncwarp();
@@ -556,15 +591,15 @@ __global__ void __launch_bounds__(MODE == kModeFp8 ? 384 : 256, 1)
             const uint32_t va = smem_u32(vs);
             const uint32_t d = tmem + 64 * m;
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              mma_bf16_ss(d, sdesc(va + kk * 2048, 16384, 1024),
-                          sdesc(pt + (kk >> 2) * (NR * 128) + (kk & 3) * 32, 16, 1024), idesc,
-                          (first && kk == 0) ? 0u : 1u);
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16_ss(d, sdesc(va + kk * 2048, 8192, 1024),
+                          sdesc(pt + h * (NR * 128) + kk * 32, 16, 1024), idesc,
+                          (first && h == 0 && kk == 0) ? 0u : 1u);
             mma_commit(&c->v_empty[slot]);
           }
           __syncwarp();
         }
-        if (lane == 0 && !stop) mma_commit(&c->o_done[b]);
+        if (lane == 0 && !stop) mma_commit(&c->o_done);
       }
       ++pi;
     }
@@ -593,30 +628,27 @@ __global__ void __launch_bounds__(MODE == kModeFp8 ? 384 : 256, 1)
         if (p.causal) limit = Ls - p.s_q + grow / p.h_q + 1;
       }
       float m_used = -INFINITY, l_sum = 0.f;
-      int last_b = 0, last_gt = -1;
+      int last_gt = -1;
       for (int k = pc.t0; k < pc.t1 && !stop; ++k, ++gt) {
         const int b = gt & 1;
+        // validity of the 128 keys of this tile for this row (bit i of word w = key 32w + i)
+        uint4 vmask;
+        if (MODE == kModeSparse) {
+          vmask.x = __ballot_sync(0xffffffffu, sparse_row(p, pc.unit, k * kTile + lane, false) >= 0);
+          vmask.y = __ballot_sync(0xffffffffu, sparse_row(p, pc.unit, k * kTile + 32 + lane, false) >= 0);
+          vmask.z = __ballot_sync(0xffffffffu, sparse_row(p, pc.unit, k * kTile + 64 + lane, false) >= 0);
+          vmask.w = __ballot_sync(0xffffffffu, sparse_row(p, pc.unit, k * kTile + 96 + lane, false) >= 0);
+        } else {
+          const int nv = dense_tile_valid(limit, k);
+          auto word = [nv](int w) {
+            const int nb = min(32, max(0, nv - 32 * w));
+            return nb >= 32 ? 0xffffffffu : ((1u << nb) - 1u);
+          };
+          vmask = make_uint4(word(0), word(1), word(2), word(3));
+        }
         if (!timed_wait(c, &c->s_full[b], (gt >> 1) & 1, p)) { stop = true; break; }
         tc_fence_after();
         const uint32_t s_addr = tmem + lane_base + kTmemS + 128 * b;
-        // validity of the 128 keys of this tile for this row
-        uint32_t vmask[4];
-        if (MODE == kModeSparse) {
-#pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            uint32_t mw = 0;
-            for (int i = 0; i < 32; ++i)
-              if (sparse_row(p, pc.unit, k * kTile + 32 * w + i, false) >= 0) mw |= 1u << i;
-            vmask[w] = mw;
-          }
-        } else {
-          const int nv = dense_tile_valid(limit, k);
-#pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            const int nb = min(32, max(0, nv - 32 * w));
-            vmask[w] = nb >= 32 ? 0xffffffffu : ((1u << nb) - 1u);
-          }
-        }
         // pass 1: tile max
         float tmax = -INFINITY;
 #pragma unroll 1
@@ -624,9 +656,10 @@ __global__ void __launch_bounds__(MODE == kModeFp8 ? 384 : 256, 1)
           uint32_t sv[32];
           tmem_ld32(s_addr + 32 * w, sv);
           tmem_ld_wait();
+          const uint32_t mw = pick4u(vmask, w);
 #pragma unroll
           for (int i = 0; i < 32; ++i)
-            if (vmask[w] & (1u << i)) tmax = fmaxf(tmax, __uint_as_float(sv[i]));
+            tmax = fmaxf(tmax, ((mw >> i) & 1u) ? __uint_as_float(sv[i]) : -INFINITY);
         }
         if (!rvalid) tmax = -INFINITY;
         float alpha = 1.f;
@@ -638,57 +671,64 @@ __global__ void __launch_bounds__(MODE == kModeFp8 ? 384 : 256, 1)
           m_used = m_new;
           l_sum *= alpha;
         }
-        if (owner) c->alpha[r] = alpha;
-        if (need) c->rescale_flag[gt & 1] = 1;
-        if (!group_sync(c, &c->grp_sm, gph, p)) { stop = true; break; }
-        const bool do_rescale = *(volatile int*)&c->rescale_flag[gt & 1] != 0;
-        if (do_rescale) {
-          // O^T of the previous tile must be complete before it is rescaled
-          const int pb = (gt - 1) & 1;
-          if (!timed_wait(c, &c->o_done[pb], ((gt - 1) >> 1) & 1, p)) { stop = true; }
-          if (!stop) {
-            tc_fence_after();
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-#pragma unroll
-              for (int c16 = 0; c16 < NR / 16; ++c16) {
-                uint32_t ov[16];
-                const uint32_t a = tmem + lane_base + 64 * m + 16 * c16;
-                tmem_ld16(a, ov);
-                tmem_ld_wait();
-#pragma unroll
-                for (int i = 0; i < 16; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * c->alpha[16 * c16 + i]);
-                tmem_st16(a, ov);
-              }
-            }
-            tmem_st_wait();
-          }
-          if (!group_sync(c, &c->grp_sm, gph, p)) stop = true;
-          if (threadIdx.x == 128) c->rescale_flag[gt & 1] = 0;
-        }
-        if (stop) break;
-        // P^T buffer b was last read by the O MMAs of tile gt-2
-        if (gt >= 2 && !timed_wait(c, &c->o_done[b], ((gt - 2) >> 1) & 1, p)) { stop = true; break; }
-        // pass 2: probabilities -> bf16 P^T (K-major [NR rows][128 tokens]), row sum
-        uint8_t* ptile = sP + b * L::pt_bytes;
+        // pass 2: probabilities (masked by select, never by branch) -> bf16, staged
+        // in TMEM over the S columns already read (tokens 32w.. -> columns 16w..)
         const float mc = (m_used == -INFINITY ? 0.f : m_used) * p.scale_log2;
+        float part = 0.f;
 #pragma unroll 1
         for (int w = 0; w < 4; ++w) {
           uint32_t sv[32];
           tmem_ld32(s_addr + 32 * w, sv);
           tmem_ld_wait();
-          if (owner && r < NR) {
-            uint32_t pk[16];
+          const uint32_t mw = rvalid ? pick4u(vmask, w) : 0u;
+          uint32_t pk[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              float p0 = (rvalid && (vmask[w] >> (2 * i)) & 1u) ? ex2_approx(__uint_as_float(sv[2 * i]) * p.scale_log2 - mc) : 0.f;
-              float p1 = (rvalid && (vmask[w] >> (2 * i + 1)) & 1u) ? ex2_approx(__uint_as_float(sv[2 * i + 1]) * p.scale_log2 - mc) : 0.f;
-              pk[i] = pack_bf16x2(p0, p1);
-              l_sum += p0 + p1;
+          for (int i = 0; i < 16; ++i) {
+            const float e0 = ex2_approx(fmaf(__uint_as_float(sv[2 * i]), p.scale_log2, -mc));
+            const float e1 = ex2_approx(fmaf(__uint_as_float(sv[2 * i + 1]), p.scale_log2, -mc));
+            const float p0 = ((mw >> (2 * i)) & 1u) ? e0 : 0.f;
+            const float p1 = ((mw >> (2 * i + 1)) & 1u) ? e1 : 0.f;
+            pk[i] = pack_bf16x2(p0, p1);
+            part += p0 + p1;
+          }
+          tmem_st16(s_addr + 16 * w, pk);
+        }
+        tmem_st_wait();
+        l_sum += part;
+        if (owner) c->alpha[r] = alpha;
+        if (need) c->rescale_flag[gt & 1] = 1;
+        if (!group_sync(c, &c->grp_sm, gph, p)) { stop = true; break; }
+        const bool do_rescale = *(volatile int*)&c->rescale_flag[gt & 1] != 0;
+        // the O MMAs of the previous tile must be complete before O^T is
+        // rescaled and before P^T (which they read) is overwritten
+        if (gt >= 1 && !timed_wait(c, &c->o_done, (gt - 1) & 1, p)) { stop = true; break; }
+        tc_fence_after();
+        if (do_rescale) {
+#pragma unroll 1
+          for (int m = 0; m < 4; ++m) {
+#pragma unroll 1
+            for (int c16 = 0; c16 < NR / 16; ++c16) {
+              uint32_t ov[16];
+              const uint32_t a = tmem + lane_base + 64 * m + 16 * c16;
+              tmem_ld16(a, ov);
+              tmem_ld_wait();
+#pragma unroll
+              for (int i = 0; i < 16; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * c->alpha[16 * c16 + i]);
+              tmem_st16(a, ov);
             }
-            // tokens 32w..32w+31 -> slice (w>>1), chunks 4*(w&1) .. +3
-            uint8_t* slice = ptile + (w >> 1) * (NR * 128);
-            uint8_t* rowp = slice + (r >> 3) * 1024 + (r & 7) * 128;
+          }
+          tmem_st_wait();
+          if (!group_sync(c, &c->grp_sm, gph, p)) { stop = true; break; }
+          if (threadIdx.x == 128) c->rescale_flag[gt & 1] = 0;
+        }
+        // P^T, K-major [NR rows][128 tokens]: tokens 64h.. in slice h, 8 tokens per 16-B chunk
+#pragma unroll 1
+        for (int w = 0; w < 4; ++w) {
+          uint32_t pk[16];
+          tmem_ld16(s_addr + 16 * w, pk);
+          tmem_ld_wait();
+          if (owner && r < NR) {
+            uint8_t* rowp = sP + (w >> 1) * (NR * 128) + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
               const int ch = 4 * (w & 1) + q;
@@ -697,16 +737,16 @@ __global__ void __launch_bounds__(MODE == kModeFp8 ? 384 : 256, 1)
             }
           }
         }
+        tc_fence_before();
+        mbar_arrive(&c->s_empty[b]);  // scores and staged probabilities of this buffer are consumed
         fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(&c->s_empty[b]);
-        mbar_arrive(&c->p_full[b]);
-        last_b = b;
+        mbar_arrive(&c->p_full);
         last_gt = gt;
       }
       if (stop) break;
       // ---------------- epilogue of the piece
-      if (last_gt >= 0 && !timed_wait(c, &c->o_done[last_b], (last_gt >> 1) & 1, p)) { stop = true; break; }
+      if (last_gt >= 0 && !timed_wait(c, &c->o_done, last_gt & 1, p)) { stop = true; break; }
       tc_fence_after();
       if (owner) {
         float inv = 0.f, lse = -INFINITY;
@@ -722,10 +762,10 @@ __global__ void __launch_bounds__(MODE == kModeFp8 ? 384 : 256, 1)
         }
       }
       if (!group_sync(c, &c->grp_sm, gph, p)) { stop = true; break; }
-#pragma unroll
+#pragma unroll 1
       for (int m = 0; m < 4; ++m) {
         const int d = 128 * m + 32 * q4 + lane;
-#pragma unroll
+#pragma unroll 1
         for (int c16 = 0; c16 < NR / 16; ++c16) {
           uint32_t ov[16];
           tmem_ld16(tmem + lane_base + 64 * m + 16 * c16, ov);
@@ -736,7 +776,8 @@ __global__ void __launch_bounds__(MODE == kModeFp8 ? 384 : 256, 1)
             if (rr < rows_here) {
               const float val = __uint_as_float(ov[i]) * c->inv_l[rr];
               if (pc.single)
-                static_cast<__nv_bfloat16*>(p.out)[((size_t)pc.unit * p.rows + row0 + rr) * kDv + d] = __float2bfloat16_rn(val);
+                static_cast<__nv_bfloat16*>(p.out)[((size_t)pc.unit * p.rows + row0 + rr) * kDv + d] =
+                    __float2bfloat16_rn(val);
               else
                 p.ws_o[((size_t)pc.ws_idx * p.rows + row0 + rr) * kDv + d] = val;
             }
@@ -758,25 +799,25 @@ __global__ void __launch_bounds__(MODE == kModeFp8 ? 384 : 256, 1)
 
 // ---------------------------------------------------------------- host side
 template <int NR, int MODE>
-static cudaError_t launch_one(const CUtensorMap& tq, const CUtensorMap& tkv, const CUtensorMap& taux,
-                              const DecodeParams& p, int parts, int row_groups, cudaStream_t stream) {
+static cudaError_t launch_one(const CUtensorMap& tq, const CUtensorMap& tkv, const DecodeParams& p, int parts,
+                              int row_groups, cudaStream_t stream) {
   constexpr int smem = Smem<NR>::total + 1024;
   auto kern = mla_decode_kernel<NR, MODE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(parts, row_groups);
-  kern<<<grid, MODE == kModeFp8 ? 384 : 256, smem, stream>>>(tq, tkv, taux, p);
+  kern<<<grid, MODE == kModeBf16 ? 256 : 320, smem, stream>>>(tq, tkv, p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_decode(int rows_per_cta, int mode, const CUtensorMap& tq, const CUtensorMap& tkv,
-                          const CUtensorMap& taux, const DecodeParams& p, int parts, int row_groups,
-                          cudaStream_t stream) {
-#define MLA_DISPATCH(NRV)                                                                              \
-  if (mode == kModeBf16) return launch_one<NRV, kModeBf16>(tq, tkv, taux, p, parts, row_groups, stream); \
-  if (mode == kModeFp8) return launch_one<NRV, kModeFp8>(tq, tkv, taux, p, parts, row_groups, stream);   \
-  return launch_one<NRV, kModeSparse>(tq, tkv, taux, p, parts, row_groups, stream);
-  if (rows_per_cta <= 16) { MLA_DISPATCH(16) }
+                          const DecodeParams& p, int parts, int row_groups, cudaStream_t stream) {
+#define MLA_DISPATCH(NRV)                                                                         \
+  if (mode == kModeBf16) return launch_one<NRV, kModeBf16>(tq, tkv, p, parts, row_groups, stream); \
+  if (mode == kModeFp8) return launch_one<NRV, kModeFp8>(tq, tkv, p, parts, row_groups, stream);   \
+  return launch_one<NRV, kModeSparse>(tq, tkv, p, parts, row_groups, stream);
+  // <= 16 rows run in the 32-row kernel: the extra P^T rows are written as
+  // zeros and their output rows are never stored
   if (rows_per_cta <= 32) { MLA_DISPATCH(32) }
   if (rows_per_cta <= 48) { MLA_DISPATCH(48) }
   MLA_DISPATCH(64)

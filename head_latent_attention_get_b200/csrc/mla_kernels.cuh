@@ -17,6 +17,7 @@ struct DecodeParams {
   const int32_t* seqlens;
   const int32_t* indices;                   // sparse mode
   const uint8_t* kcache_fp8;                // FP8 mode: token records
+  const void* kcache;                       // cache base (L2 prefetch, sparse gather)
   const int32_t* tile_md;
   const int32_t* split_ptr;
   void* out;                                // bf16 [units*rows][512]
@@ -29,8 +30,7 @@ struct DecodeParams {
 };
 
 cudaError_t launch_decode(int rows_per_cta, int mode, const CUtensorMap& tq, const CUtensorMap& tkv,
-                          const CUtensorMap& taux, const DecodeParams& p, int parts, int row_groups,
-                          cudaStream_t stream);
+                          const DecodeParams& p, int parts, int row_groups, cudaStream_t stream);
 mla_status_t launch_metadata(const int32_t* seqlens, int U, int topk, int parts, int32_t* tile_md,
                              int32_t* num_splits, cudaStream_t stream);
 mla_status_t launch_combine(const void* workspace, int units, int rows, int parts, const int32_t* split_ptr,

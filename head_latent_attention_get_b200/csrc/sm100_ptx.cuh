@@ -1,5 +1,5 @@
 // Thin inline-PTX wrappers for the sm_100a features the decode kernels use:
-// mbarriers (with bounded waits), TMA tile / gather4 loads, TMEM allocation,
+// mbarriers (with bounded waits), TMA tile loads, cp.async, TMEM allocation,
 // tcgen05.mma (kind::f16, bf16 inputs, fp32 accumulate), tcgen05.commit and
 // tcgen05.ld / tcgen05.st, plus the shared-memory and instruction descriptors.
 //
@@ -93,15 +93,24 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
       : "memory");
 }
-// 2-D load of four arbitrary rows (tensor map box is one row high).
-__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y0,
-                                            int y1, int y2, int y3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y0), "r"(y1), "r"(y2),
-      "r"(y3)
-      : "memory");
+// Bulk prefetch of a contiguous global range into L2 (no shared memory used).
+__device__ __forceinline__ void prefetch_l2(const void* gmem, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(gmem)), "r"(bytes)
+               : "memory");
+}
+
+// 16-byte asynchronous global->shared copy (Ampere cp.async, L2-only caching).
+// src_bytes < 16 zero-fills the rest of the 16 bytes; 0 reads nothing.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// Waits until at most N of this thread's committed cp.async groups are pending.
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 // ---------------------------------------------------------------- TMEM
