@@ -116,8 +116,12 @@ mla_status_t run_decode(const mla_decode_args* a, const int32_t* indices, int to
   p.debug_flags = a->debug_flags;
   const int row_groups = (rows + kRowsPerCta - 1) / kRowsPerCta;
   const int rows_per_cta = rows < kRowsPerCta ? rows : kRowsPerCta;
-  if (launch_decode(rows_per_cta, mode, tq, tkv, p, a->num_sm_parts, row_groups, stream) != cudaSuccess)
-    return MLA_ERR_CUDA;
+  // more than 64 rows on the BF16 paged cache: one CTA pair per part shares each
+  // cache tile between the two row halves instead of loading it twice
+  const cudaError_t e = (mode == kModeBf16 && row_groups == 2)
+                            ? launch_decode_pair(tq, tkv, p, a->num_sm_parts, stream)
+                            : launch_decode(rows_per_cta, mode, tq, tkv, p, a->num_sm_parts, row_groups, stream);
+  if (e != cudaSuccess) return MLA_ERR_CUDA;
   if (a->debug_flags & MLA_DEBUG_SKIP_COMBINE) return MLA_OK;
   return launch_combine(a->workspace, U, rows, a->num_sm_parts, a->num_splits, a->out, a->lse, stream);
 }
@@ -148,7 +152,16 @@ mla_status_t mla_get_num_sm_parts(int device, int s_q, int h_q, int h_kv, int to
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || sms <= 0)
     return MLA_ERR_CUDA;
   const int groups = (rows + kRowsPerCta - 1) / kRowsPerCta;
-  *num_sm_parts = sms / groups > 0 ? sms / groups : 1;
+  int parts = sms / groups > 0 ? sms / groups : 1;
+  if (groups == 2) {  // two CTAs per part: no more parts than CTA pairs that fit at once
+    int cur = 0;
+    if (cudaGetDevice(&cur) != cudaSuccess) return MLA_ERR_CUDA;
+    if (cur != device && cudaSetDevice(device) != cudaSuccess) return MLA_ERR_CUDA;
+    const int fit = max_pair_clusters();
+    if (cur != device) cudaSetDevice(cur);
+    if (fit > 0 && fit < parts) parts = fit;
+  }
+  *num_sm_parts = parts;
   return MLA_OK;
 }
 

@@ -1,0 +1,558 @@
+// MLA decode for units with more than 64 query rows (e.g. 128 heads), BF16
+// paged cache: one CTA pair (cluster of 2 CTAs on two SMs) per scheduler part.
+//
+// Same computation as mla_decode.cu -- per unit, softmax(scale * Q K^T) V with
+// K = the 576-dim latent row and V = its first 512 dims ([flashinfer] ...
+// NVFP4 DeepSeek-V4 decoding, README section; FlashMLA-ETAP summary, core
+// mechanism) -- organised so that a 128-row unit is served by two SMs that
+// share every cache byte instead of each reading all of it:
+//
+//   step = two consecutive 128-token tiles (256 tokens); CTA r loads
+//          K of tile r (all 576 dims) and V of all 256 tokens for its value
+//          dims {256j + 128r + [0,128) : j = 0,1}.
+//   S = Q K^T   pair MMA M=128 (64 rows per CTA) x N=256 (128 tokens per CTA)
+//               x K=576. Each CTA's TMEM receives its 64 rows x 256 tokens:
+//               lanes 0-63 hold tokens 0-127, lanes 64-127 tokens 128-255.
+//   softmax     thread (row, half) of the CTA reads its row's 128 scores of
+//               token half `half`; the row max is agreed between the two
+//               threads of a row through shared memory, once per step.
+//   O = P V     pair MMA M=128 x N=256 (value dims, 128 per CTA) x K=256
+//               tokens, twice (dims 0-255 and 256-511). P is this CTA's 64
+//               rows (K-major, written by the softmax threads); V is read
+//               MN-major straight from the token-major cache rows. O stays in
+//               this CTA's TMEM (rows on lanes), so rescaling is thread-local.
+// TMEM per CTA: O 2 x 128 columns + S 2 x 128 columns = 512.
+//
+// Warp roles (256 threads per CTA):
+//   0 Q + K slices via TMA (both CTAs; completion counted on the even CTA's barriers)
+//   1 TMEM allocation (both) and S MMA issue (even CTA)
+//   2 O MMA issue (even CTA)
+//   3 V slots via TMA (both)
+//   4-7 softmax + epilogue (both): thread i = (row i % 64, token half i / 64)
+// All waits are bounded; a timeout sets MLA_DEVICE_STATUS_TIMEOUT, raises the
+// abort flag of both CTAs, and every role winds down to the final cluster
+// barrier, which both CTAs always reach.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "mla_decode_util.cuh"
+
+namespace mla {
+namespace pair {
+
+constexpr int kNK = 3;               // K ring: 128 tokens x 64 dims (16 KB)
+constexpr int kNV = 4;               // V ring: 64 tokens x 128 value dims (two 8 KB halves)
+constexpr int kSlot = 16384;
+constexpr int kQBytes = 9 * 8192;    // 64 rows x 576 dims
+constexpr int kPBytes = 4 * 8192;    // 64 rows x 256 tokens
+constexpr int kPrefetchSteps = 2;    // L2 prefetch distance
+constexpr int kTmemCols = 512;
+constexpr int kTmemS = 256;          // S buffers at columns 256 and 384; O at 0 and 128
+constexpr float kRescaleLog2 = 8.0f;
+
+struct Smem {
+  static constexpr int q = 0;
+  static constexpr int k = q + kQBytes;
+  static constexpr int v = k + kNK * kSlot;
+  static constexpr int pt = v + kNV * kSlot;
+  static constexpr int ctrl = pt + kPBytes;
+  static constexpr int total = ctrl + 2048;
+};
+
+struct Ctrl {
+  // barriers counted on the even CTA (the MMA issuer) ...
+  uint64_t q_full;                     // 1 arrival (+ both CTAs' Q bytes)
+  uint64_t k_full[kNK];                // 1 arrival (+ both CTAs' K bytes)
+  uint64_t v_full[kNV];                // 2 arrivals, one per CTA (+ bytes)
+  uint64_t s_empty[2], p_full, o_free; // 8 arrivals: 4 softmax warps x 2 CTAs
+  uint64_t drain_s, drain_o;
+  // ... and in each CTA
+  uint64_t q_empty, k_empty[kNK], v_empty[kNV];  // pair-MMA commits
+  uint64_t s_full[2], o_done;                    // pair-MMA commits
+  uint64_t v_fix;                                // local loads of partial pages
+  uint64_t grp_sm;                               // 128 softmax threads
+  uint32_t tmem_base;
+  int abort_flag;
+  float mx[2][2][64];                  // [step parity][token half][row]: per-half tile max
+  float lx[2][64];                     // [token half][row]: per-half row sum
+};
+static_assert(sizeof(Ctrl) <= 2048, "control block");
+
+struct Pair {
+  uint32_t rank;
+  bool leader;
+  Ctrl* c;
+  uint32_t peer_abort;                 // cluster address of the other CTA's abort flag
+};
+
+__device__ __forceinline__ void raise_abort(const Pair& pr, const DecodeParams& p) {
+  atomicOr(p.status, (uint32_t)MLA_DEVICE_STATUS_TIMEOUT);
+  *(volatile int*)&pr.c->abort_flag = 1;
+  st_cluster_u32(pr.peer_abort, 1u);
+}
+
+__device__ __forceinline__ bool aborted(const Pair& pr) { return *(volatile int*)&pr.c->abort_flag != 0; }
+
+// Bounded wait with cluster-scope acquire (several barriers receive arrivals
+// from the other CTA or pair-MMA commits).
+__device__ __forceinline__ bool pwait(const Pair& pr, uint64_t* bar, uint32_t parity, const DecodeParams& p) {
+  if (aborted(pr)) return false;
+  if (mbar_wait_cluster(bar, parity, p.timeout_ns)) return true;
+  raise_abort(pr, p);
+  return false;
+}
+
+__device__ __forceinline__ bool group_sync(const Pair& pr, uint32_t& phase, const DecodeParams& p) {
+  mbar_arrive(&pr.c->grp_sm);
+  const bool ok = pwait(pr, &pr.c->grp_sm, phase & 1, p);
+  ++phase;
+  return ok;
+}
+
+// Arrive on barrier `bar` of the even CTA (a local arrive there, a remote one from the odd CTA).
+__device__ __forceinline__ void arrive_leader(const Pair& pr, uint64_t* bar) {
+  mbar_arrive_cluster(map_to_rank(smem_u32(bar), 0));
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
+    mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
+                           const DecodeParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem + Smem::q;
+  uint8_t* sK = smem + Smem::k;
+  uint8_t* sV = smem + Smem::v;
+  uint8_t* sP = smem + Smem::pt;
+  Ctrl* c = reinterpret_cast<Ctrl*>(smem + Smem::ctrl);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  Pair pr;
+  pr.rank = cluster_rank();
+  pr.leader = pr.rank == 0;
+  pr.c = c;
+  pr.peer_abort = map_to_rank(smem_u32(&c->abort_flag), pr.rank ^ 1u);
+  const int part = blockIdx.x >> 1;
+  const int row0 = 64 * (int)pr.rank;   // first row of this CTA within a unit
+
+  if (threadIdx.x == 0) {
+    mbar_init(&c->q_full, 1);
+    for (int i = 0; i < kNK; ++i) mbar_init(&c->k_full[i], 1);
+    for (int i = 0; i < kNV; ++i) mbar_init(&c->v_full[i], 2);
+    for (int i = 0; i < 2; ++i) mbar_init(&c->s_empty[i], 8);
+    mbar_init(&c->p_full, 8);
+    mbar_init(&c->o_free, 8);
+    mbar_init(&c->drain_s, 1);
+    mbar_init(&c->drain_o, 1);
+    mbar_init(&c->q_empty, 1);
+    for (int i = 0; i < kNK; ++i) mbar_init(&c->k_empty[i], 1);
+    for (int i = 0; i < kNV; ++i) mbar_init(&c->v_empty[i], 1);
+    for (int i = 0; i < 2; ++i) mbar_init(&c->s_full[i], 1);
+    mbar_init(&c->o_done, 1);
+    mbar_init(&c->v_fix, 1);
+    mbar_init(&c->grp_sm, 128);
+    c->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_kv);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(&c->tmem_base, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();  // barriers initialised and TMEM allocated in both CTAs
+  tc_fence_after();
+  const uint32_t tmem = c->tmem_base;
+
+  PieceIter it;
+  it.init(p, part);
+  Piece pc;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ Q + K slices
+    int kc = 0, pi = 0, q_issued = 0;
+    bool stop = false;
+    while (!stop && it.next(pc)) {
+      if (lane == 0) {
+        if (!pwait(pr, &c->q_empty, (pi & 1) ^ 1, p)) {
+          stop = true;
+        } else {
+          const uint32_t qbar = map_to_rank(smem_u32(&c->q_full), 0);
+          if (pr.leader) mbar_arrive_expect_tx(&c->q_full, 2 * kQBytes);
+          const int qy = pc.unit * p.rows + row0;
+          for (int j = 0; j < 9; ++j) tma_load_2d_pair(sQ + j * 8192, &tm_q, qbar, 64 * j, qy);
+          ++q_issued;
+        }
+        const int req = pc.unit;
+        const int npg = (p.seqlens[req] + kPage - 1) / kPage;
+        for (int k = pc.t0; k < pc.t1 && !stop; k += 2) {
+          // own tile; past the piece's end the pair's other tile is loaded again (its keys are masked)
+          const int t = (k + (int)pr.rank < pc.t1) ? k + (int)pr.rank : k;
+          int pa = page_of(p, req, 2 * t, npg);
+          int pb = page_of(p, req, 2 * t + 1, npg);
+          if (pb < 0) pb = pa;
+          const int tp = t + 2 * kPrefetchSteps;
+          if (tp < pc.t1) {
+            for (int h = 0; h < 2; ++h) {
+              const int pf = page_of(p, req, 2 * tp + h, npg);
+              if (pf >= 0)
+                prefetch_l2(static_cast<const uint8_t*>(p.kcache) + (size_t)pf * kPage * kDqk * 2, kPage * kDqk * 2);
+            }
+          }
+          for (int j = 0; j < 9; ++j, ++kc) {
+            const int slot = kc % kNK;
+            uint8_t* dst = sK + slot * kSlot;
+            if (!pwait(pr, &c->k_empty[slot], ((kc / kNK) & 1) ^ 1, p)) { stop = true; break; }
+            const uint32_t kbar = map_to_rank(smem_u32(&c->k_full[slot]), 0);
+            if (pr.leader) mbar_arrive_expect_tx(&c->k_full[slot], 2 * kSlot);
+            tma_load_2d_pair(dst, &tm_kv, kbar, 64 * j, pa * kPage);
+            tma_load_2d_pair(dst + 8192, &tm_kv, kbar, 64 * j, pb * kPage);
+          }
+        }
+      }
+      stop = __shfl_sync(0xffffffffu, stop ? 1 : 0, 0) != 0;
+      ++pi;
+    }
+    if (lane == 0 && pr.leader) {  // the even CTA's barriers count both CTAs' copies
+      if (q_issued > 0) mbar_wait_cluster(&c->q_full, (uint32_t)((q_issued - 1) & 1), p.timeout_ns);
+      for (int i = kc > kNK ? kc - kNK : 0; i < kc; ++i)
+        mbar_wait_cluster(&c->k_full[i % kNK], (uint32_t)((i / kNK) & 1), p.timeout_ns);
+    }
+    __syncwarp();
+  } else if (warp == 3) {
+    // ------------------------------------------------------------ V slots
+    // slot (q, jd): page q of the step (tile k + q/2, page half q%2), value
+    // dims 256*jd + 128*rank + [0,128) as two 64-dim halves.
+    int vc = 0, fixc = 0;
+    bool stop = false;
+    while (!stop && it.next(pc)) {
+      const int req = pc.unit;
+      const int Ls = p.seqlens[req];
+      const int npg = (Ls + kPage - 1) / kPage;
+      for (int k = pc.t0; k < pc.t1 && !stop; k += 2) {
+        for (int q = 0; q < 4 && !stop; ++q) {
+          const int tile = k + (q >> 1), pj = 2 * tile + (q & 1);
+          const int nv = tile < pc.t1 ? max(0, min(kPage, Ls - kPage * pj)) : 0;
+          const int pg = nv > 0 ? page_of(p, req, pj, npg) : 0;
+          for (int jd = 0; jd < 2; ++jd, ++vc) {
+            const int slot = vc % kNV;
+            uint8_t* dst = sV + slot * kSlot;
+            bool ok = true;
+            if (lane == 0) ok = pwait(pr, &c->v_empty[slot], ((vc / kNV) & 1) ^ 1, p);
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok) { stop = true; break; }
+            const int x0 = 256 * jd + 128 * (int)pr.rank;
+            if (nv == kPage) {
+              if (lane == 0) {
+                const uint32_t vbar = map_to_rank(smem_u32(&c->v_full[slot]), 0);
+                if (pr.leader) mbar_arrive_expect_tx(&c->v_full[slot], 2 * kSlot);
+                else mbar_arrive_cluster(vbar);
+                tma_load_2d_pair(dst, &tm_kv, vbar, x0, pg * kPage);
+                tma_load_2d_pair(dst + 8192, &tm_kv, vbar, x0 + 64, pg * kPage);
+              }
+            } else {
+              // keys past the request's end have zero probability, but their
+              // cache rows may hold anything (0 x NaN = NaN): load locally,
+              // zero those rows, then count the slot as full
+              if (nv > 0) {
+                if (lane == 0) {
+                  mbar_arrive_expect_tx(&c->v_fix, kSlot);
+                  tma_load_2d(dst, &tm_kv, &c->v_fix, x0, pg * kPage);
+                  tma_load_2d(dst + 8192, &tm_kv, &c->v_fix, x0 + 64, pg * kPage);
+                  ok = pwait(pr, &c->v_fix, fixc & 1, p);
+                }
+                ++fixc;
+                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                if (!ok) { stop = true; break; }
+              }
+              const uint4 z = make_uint4(0, 0, 0, 0);
+              for (int i = nv * 8 + lane; i < kPage * 8; i += 32) {  // 8 chunks of 16 B per 128-B row
+                *reinterpret_cast<uint4*>(dst + i * 16) = z;
+                *reinterpret_cast<uint4*>(dst + 8192 + i * 16) = z;
+              }
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) arrive_leader(pr, &c->v_full[slot]);
+            }
+          }
+        }
+      }
+    }
+    if (lane == 0 && pr.leader)
+      for (int i = vc > kNV ? vc - kNV : 0; i < vc; ++i)
+        mbar_wait_cluster(&c->v_full[i % kNV], (uint32_t)((i / kNV) & 1), p.timeout_ns);
+    __syncwarp();
+  } else if (warp == 1 && pr.leader) {
+    // ------------------------------------------------------------ S issuer
+    const uint32_t idesc = idesc_bf16(128, 256, false, false);
+    int kc = 0, gt = 0, pi = 0;
+    bool stop = false;
+    if (lane == 0) {
+      while (!stop && it.next(pc)) {
+        if (!pwait(pr, &c->q_full, pi & 1, p)) { stop = true; break; }
+        for (int k = pc.t0; k < pc.t1 && !stop; k += 2, ++gt) {
+          const int b = gt & 1;
+          if (!pwait(pr, &c->s_empty[b], ((gt >> 1) & 1) ^ 1, p)) { stop = true; break; }
+          tc_fence_after();
+          const uint32_t d = tmem + kTmemS + 128 * b;
+          for (int j = 0; j < 9; ++j, ++kc) {
+            const int slot = kc % kNK;
+            if (!pwait(pr, &c->k_full[slot], (kc / kNK) & 1, p)) { stop = true; break; }
+            tc_fence_after();
+            const uint32_t qa = smem_u32(sQ + j * 8192), kb = smem_u32(sK + slot * kSlot);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16_ss_pair(d, sdesc(qa + kk * 32, 16, 1024), sdesc(kb + kk * 32, 16, 1024), idesc,
+                               (j | kk) != 0 ? 1u : 0u);
+            mma_commit_pair(&c->k_empty[slot]);
+          }
+          if (!stop && !(gt == 0 && (p.debug_flags & MLA_DEBUG_WITHHOLD_SCORES))) mma_commit_pair(&c->s_full[b]);
+        }
+        if (!stop) mma_commit_pair(&c->q_empty);
+        ++pi;
+      }
+      mma_commit_pair(&c->drain_s);  // every MMA this thread issued has completed before teardown
+      mbar_wait(&c->drain_s, 0, p.timeout_ns);
+    }
+    __syncwarp();
+  } else if (warp == 2 && pr.leader) {
+    // ------------------------------------------------------------ O issuer
+    const uint32_t idesc = idesc_bf16(128, 256, false, true);
+    int vc = 0, gt = 0, pi = 0;
+    bool stop = false;
+    if (lane == 0) {
+      while (!stop && it.next(pc)) {
+        for (int k = pc.t0; k < pc.t1 && !stop; k += 2, ++gt) {
+          const bool first = (k == pc.t0);
+          if (first && pi > 0 && !pwait(pr, &c->o_free, (pi - 1) & 1, p)) { stop = true; break; }
+          if (!pwait(pr, &c->p_full, gt & 1, p)) { stop = true; break; }
+          const uint32_t pt = smem_u32(sP);
+          for (int q = 0; q < 4 && !stop; ++q) {
+            for (int jd = 0; jd < 2; ++jd, ++vc) {
+              const int slot = vc % kNV;
+              if (!pwait(pr, &c->v_full[slot], (vc / kNV) & 1, p)) { stop = true; break; }
+              tc_fence_after();
+              const uint32_t va = smem_u32(sV + slot * kSlot);
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                mma_bf16_ss_pair(tmem + 128 * jd, sdesc(pt + q * 8192 + kk * 32, 16, 1024),
+                                 sdesc(va + kk * 2048, 8192, 1024), idesc, (first && q == 0 && kk == 0) ? 0u : 1u);
+              mma_commit_pair(&c->v_empty[slot]);
+            }
+          }
+          if (!stop) mma_commit_pair(&c->o_done);
+        }
+        ++pi;
+      }
+      mma_commit_pair(&c->drain_o);
+      mbar_wait(&c->drain_o, 0, p.timeout_ns);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int ti = threadIdx.x - 128;                     // TMEM lane of this thread
+    const int row = ti & 63, half = ti >> 6;
+    const int grow = row0 + row;                          // row within the unit
+    const bool rvalid = grow < p.rows;
+    const uint32_t lane_base = (uint32_t)(32 * (warp - 4)) << 16;
+    const float thresh = kRescaleLog2 / p.scale_log2;     // raw-score units
+    uint32_t gph = 0;
+    int gt = 0;
+    bool stop = false;
+    while (!stop && it.next(pc)) {
+      const int req = pc.unit;
+      const int Ls = p.seqlens[req];
+      const int limit = p.causal ? Ls - p.s_q + grow / p.h_q + 1 : Ls;
+      float m_used = -INFINITY, l_sum = 0.f;
+      int last_gt = -1;
+      for (int k = pc.t0; k < pc.t1 && !stop; k += 2, ++gt) {
+        const int b = gt & 1;
+        const int tile = k + half;
+        const int nv = (rvalid && tile < pc.t1) ? dense_tile_valid(limit, tile) : 0;
+        if (!pwait(pr, &c->s_full[b], (gt >> 1) & 1, p)) { stop = true; break; }
+        tc_fence_after();
+        const uint32_t s_addr = tmem + lane_base + kTmemS + 128 * b;
+        // pass 1: max over this thread's 128 keys
+        float tmax = -INFINITY;
+#pragma unroll 1
+        for (int w = 0; w < 4; ++w) {
+          uint32_t sv[32];
+          tmem_ld32(s_addr + 32 * w, sv);
+          tmem_ld_wait();
+          const int nb = min(32, max(0, nv - 32 * w));
+#pragma unroll
+          for (int i = 0; i < 32; ++i) tmax = fmaxf(tmax, i < nb ? __uint_as_float(sv[i]) : -INFINITY);
+        }
+        c->mx[gt & 1][half][row] = tmax;
+        if (!group_sync(pr, gph, p)) { stop = true; break; }
+        tmax = fmaxf(tmax, c->mx[gt & 1][half ^ 1][row]);
+        // both threads of a row take the same decision from the same values
+        float alpha = 1.f;
+        bool need = false;
+        if (tmax > m_used + thresh || (m_used == -INFINITY && tmax > -INFINITY)) {
+          alpha = (m_used == -INFINITY) ? 0.f : ex2_approx((m_used - tmax) * p.scale_log2);
+          need = (k != pc.t0) && (m_used != -INFINITY);
+          m_used = tmax;
+          l_sum *= alpha;
+        }
+        // pass 2: probabilities (masked by select) -> bf16 staged in TMEM over
+        // the S columns already read (keys 32w.. -> columns 16w..)
+        const float mc = (m_used == -INFINITY ? 0.f : m_used) * p.scale_log2;
+        float part = 0.f;
+#pragma unroll 1
+        for (int w = 0; w < 4; ++w) {
+          uint32_t sv[32];
+          tmem_ld32(s_addr + 32 * w, sv);
+          tmem_ld_wait();
+          const int nb = min(32, max(0, nv - 32 * w));
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float e0 = ex2_approx(fmaf(__uint_as_float(sv[2 * i]), p.scale_log2, -mc));
+            const float e1 = ex2_approx(fmaf(__uint_as_float(sv[2 * i + 1]), p.scale_log2, -mc));
+            const float p0 = (2 * i < nb) ? e0 : 0.f;
+            const float p1 = (2 * i + 1 < nb) ? e1 : 0.f;
+            pk[i] = pack_bf16x2(p0, p1);
+            part += p0 + p1;
+          }
+          tmem_st16(s_addr + 16 * w, pk);
+        }
+        tmem_st_wait();
+        l_sum += part;
+        // O MMAs of the previous step must be complete before O is rescaled
+        // and before P (which they read) is overwritten
+        if (gt >= 1 && !pwait(pr, &c->o_done, (gt - 1) & 1, p)) { stop = true; break; }
+        tc_fence_after();
+        if (need) {
+#pragma unroll 1
+          for (int c16 = 0; c16 < 16; ++c16) {  // 2 x 128 columns of this row
+            uint32_t ov[16];
+            const uint32_t a = tmem + lane_base + 16 * c16;
+            tmem_ld16(a, ov);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+            tmem_st16(a, ov);
+          }
+          tmem_st_wait();
+        }
+        // P, K-major [64 rows][64 keys] per slice: keys 64s.. in slice s; this
+        // thread's keys are 128*half + [0,128), slices 2*half and 2*half + 1
+#pragma unroll 1
+        for (int w = 0; w < 4; ++w) {
+          uint32_t pk[16];
+          tmem_ld16(s_addr + 16 * w, pk);
+          tmem_ld_wait();
+          uint8_t* rowp = sP + (2 * half + (w >> 1)) * 8192 + (row >> 3) * 1024 + (row & 7) * 128;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int ch = 4 * (w & 1) + q;
+            *reinterpret_cast<uint4*>(rowp + ((ch ^ (row & 7)) << 4)) =
+                make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+          }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          arrive_leader(pr, &c->s_empty[b]);  // scores and staged probabilities consumed
+          arrive_leader(pr, &c->p_full);
+        }
+        last_gt = gt;
+      }
+      if (stop) break;
+      // ---------------- epilogue of the piece
+      c->lx[half][row] = l_sum;
+      if (!group_sync(pr, gph, p)) { stop = true; break; }
+      const float l_tot = l_sum + c->lx[half ^ 1][row];
+      if (last_gt >= 0 && !pwait(pr, &c->o_done, last_gt & 1, p)) { stop = true; break; }
+      tc_fence_after();
+      float inv = 0.f, lse = -INFINITY;
+      if (l_tot > 0.f) {
+        inv = 1.f / l_tot;
+        lse = m_used * p.scale + logf(l_tot);
+      }
+      const size_t orow = (size_t)pc.unit * p.rows + grow;
+      if (rvalid && half == 0) {
+        if (pc.single) p.lse[orow] = lse;
+        else p.ws_lse[(size_t)pc.ws_idx * p.rows + grow] = lse;
+      }
+#pragma unroll 1
+      for (int jd = 0; jd < 2; ++jd) {
+        const int d0 = 256 * jd + 128 * half;
+#pragma unroll 1
+        for (int c16 = 0; c16 < 8; ++c16) {
+          uint32_t ov[16];
+          tmem_ld16(tmem + lane_base + 128 * jd + 16 * c16, ov);
+          tmem_ld_wait();
+          if (rvalid) {
+            if (pc.single) {
+              uint32_t pk[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                pk[i] = pack_bf16x2(__uint_as_float(ov[2 * i]) * inv, __uint_as_float(ov[2 * i + 1]) * inv);
+              uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + orow * kDv + d0 + 16 * c16);
+              dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            } else {
+              float4* dst = reinterpret_cast<float4*>(p.ws_o + ((size_t)pc.ws_idx * p.rows + grow) * kDv + d0 + 16 * c16);
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                dst[i] = make_float4(__uint_as_float(ov[4 * i]) * inv, __uint_as_float(ov[4 * i + 1]) * inv,
+                                     __uint_as_float(ov[4 * i + 2]) * inv, __uint_as_float(ov[4 * i + 3]) * inv);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) arrive_leader(pr, &c->o_free);
+    }
+  }
+
+  // ---------------------------------------------------------------- teardown
+  // Copies this CTA issued whose completion is counted on the other CTA's
+  // barrier cannot be waited for here; after an abort give them time to land.
+  if (aborted(pr)) __nanosleep(100000);
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // no pair MMA, copy or remote arrive of either CTA is still pending
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem, kTmemCols);
+}
+
+}  // namespace pair
+
+cudaError_t launch_decode_pair(const CUtensorMap& tq, const CUtensorMap& tkv, const DecodeParams& p, int parts,
+                               cudaStream_t stream) {
+  constexpr int smem = pair::Smem::total + 1024;
+  auto kern = pair::mla_decode_pair_kernel;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  kern<<<2 * parts, 256, smem, stream>>>(tq, tkv, p);
+  return cudaGetLastError();
+}
+
+int max_pair_clusters() {
+  constexpr int smem = pair::Smem::total + 1024;
+  auto kern = pair::mla_decode_pair_kernel;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2, 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = 2;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) return 0;
+  return n;
+}
+
+}  // namespace mla
