@@ -15,19 +15,24 @@
 //               lanes 0-63 hold tokens 0-127, lanes 64-127 tokens 128-255.
 //   softmax     thread (row, half) of the CTA reads its row's 128 scores of
 //               token half `half`; the row max is agreed between the two
-//               threads of a row through shared memory, once per step.
+//               threads of a row through shared memory, once per step. The
+//               probabilities go straight to one of two P buffers.
 //   O = P V     pair MMA M=128 x N=256 (value dims, 128 per CTA) x K=256
 //               tokens, twice (dims 0-255 and 256-511). P is this CTA's 64
-//               rows (K-major, written by the softmax threads); V is read
-//               MN-major straight from the token-major cache rows. O stays in
-//               this CTA's TMEM (rows on lanes), so rescaling is thread-local.
+//               rows (K-major); V is read MN-major straight from the
+//               token-major cache rows. O stays in this CTA's TMEM (rows on
+//               lanes), so rescaling is thread-local.
 // TMEM per CTA: O 2 x 128 columns + S 2 x 128 columns = 512.
 //
+// Loads: one ring of 16 KB slots filled by TMA in exactly the order the MMA
+// issuer consumes them -- K of step 0, then per step g: K of step g+1, V of
+// step g -- so whichever product is being issued sees the whole ring as
+// look-ahead. The MMA issuer follows the same order: S(0), S(1), O(0), S(2),
+// O(1), ...
+//
 // Warp roles (256 threads per CTA):
-//   0 Q + K slices via TMA (both CTAs; completion counted on the even CTA's barriers)
-//   1 TMEM allocation (both) and S MMA issue (even CTA)
-//   2 O MMA issue (even CTA)
-//   3 V slots via TMA (both)
+//   0 Q, K and V via TMA (both CTAs; completion counted on the even CTA's barriers)
+//   1 TMEM allocation (both) and MMA issue (even CTA)
 //   4-7 softmax + epilogue (both): thread i = (row i % 64, token half i / 64)
 // All waits are bounded; a timeout sets MLA_DEVICE_STATUS_TIMEOUT, raises the
 // abort flag of both CTAs, and every role winds down to the final cluster
@@ -40,11 +45,12 @@
 namespace mla {
 namespace pair {
 
-constexpr int kNK = 3;               // K ring: 128 tokens x 64 dims (16 KB)
-constexpr int kNV = 4;               // V ring: 64 tokens x 128 value dims (two 8 KB halves)
+constexpr int kN = 5;                // ring slots of 16 KB: a K slice (128 tokens x 64 dims)
+                                     // or a V slot (64 tokens x 128 value dims, two 8 KB halves)
 constexpr int kSlot = 16384;
+constexpr int kThreads = 256;
 constexpr int kQBytes = 9 * 8192;    // 64 rows x 576 dims
-constexpr int kPBytes = 4 * 8192;    // 64 rows x 256 tokens
+constexpr int kPBytes = 4 * 8192;    // 64 rows x 256 tokens, per buffer
 constexpr int kPrefetchSteps = 2;    // L2 prefetch distance
 constexpr int kTmemCols = 512;
 constexpr int kTmemS = 256;          // S buffers at columns 256 and 384; O at 0 and 128
@@ -52,25 +58,23 @@ constexpr float kRescaleLog2 = 8.0f;
 
 struct Smem {
   static constexpr int q = 0;
-  static constexpr int k = q + kQBytes;
-  static constexpr int v = k + kNK * kSlot;
-  static constexpr int pt = v + kNV * kSlot;
-  static constexpr int ctrl = pt + kPBytes;
+  static constexpr int ring = q + kQBytes;
+  static constexpr int pt = ring + kN * kSlot;
+  static constexpr int ctrl = pt + 2 * kPBytes;
   static constexpr int total = ctrl + 2048;
 };
 
 struct Ctrl {
   // barriers counted on the even CTA (the MMA issuer) ...
   uint64_t q_full;                     // 1 arrival (+ both CTAs' Q bytes)
-  uint64_t k_full[kNK];                // 1 arrival (+ both CTAs' K bytes)
-  uint64_t v_full[kNV];                // 2 arrivals, one per CTA (+ bytes)
-  uint64_t s_empty[2], p_full, o_free; // 8 arrivals: 4 softmax warps x 2 CTAs
-  uint64_t drain_s, drain_o;
+  uint64_t full[kN];                   // 1 arrival (+ both CTAs' bytes of the slot)
+  uint64_t s_empty[2], p_full[2], o_free;  // 8 arrivals: 4 softmax warps x 2 CTAs
+  uint64_t drain;
   // ... and in each CTA
-  uint64_t q_empty, k_empty[kNK], v_empty[kNV];  // pair-MMA commits
-  uint64_t s_full[2], o_done;                    // pair-MMA commits
-  uint64_t v_fix;                                // local loads of partial pages
-  uint64_t grp_sm;                               // 128 softmax threads
+  uint64_t q_empty, empty[kN];         // pair-MMA commits
+  uint64_t s_full[2], o_done[2];       // pair-MMA commits; o_done[g & 1] completes O of step g
+  uint64_t v_fix;                      // local loads of partial pages
+  uint64_t grp_sm;                     // 128 softmax threads
   uint32_t tmem_base;
   int abort_flag;
   float mx[2][2][64];                  // [step parity][token half][row]: per-half tile max
@@ -114,14 +118,19 @@ __device__ __forceinline__ void arrive_leader(const Pair& pr, uint64_t* bar) {
   mbar_arrive_cluster(map_to_rank(smem_u32(bar), 0));
 }
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
+// Ring order of a piece of n steps: h = 0 -> K of step 0; h = 2g+1 -> K of
+// step g+1 (only if g+1 < n); h = 2g+2 -> V of step g.
+__device__ __forceinline__ bool ring_entry_exists(int h, int nsteps) { return !((h & 1) && (h >> 1) + 1 >= nsteps); }
+__device__ __forceinline__ bool ring_entry_is_k(int h) { return h == 0 || (h & 1); }
+__device__ __forceinline__ int ring_entry_step(int h) { return h == 0 ? 0 : (h & 1) ? (h >> 1) + 1 : (h >> 1) - 1; }
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
                            const DecodeParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + Smem::q;
-  uint8_t* sK = smem + Smem::k;
-  uint8_t* sV = smem + Smem::v;
+  uint8_t* sRing = smem + Smem::ring;
   uint8_t* sP = smem + Smem::pt;
   Ctrl* c = reinterpret_cast<Ctrl*>(smem + Smem::ctrl);
 
@@ -136,18 +145,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&c->q_full, 1);
-    for (int i = 0; i < kNK; ++i) mbar_init(&c->k_full[i], 1);
-    for (int i = 0; i < kNV; ++i) mbar_init(&c->v_full[i], 2);
-    for (int i = 0; i < 2; ++i) mbar_init(&c->s_empty[i], 8);
-    mbar_init(&c->p_full, 8);
+    for (int i = 0; i < kN; ++i) mbar_init(&c->full[i], 1);
+    for (int i = 0; i < 2; ++i) { mbar_init(&c->s_empty[i], 8); mbar_init(&c->p_full[i], 8); }
     mbar_init(&c->o_free, 8);
-    mbar_init(&c->drain_s, 1);
-    mbar_init(&c->drain_o, 1);
+    mbar_init(&c->drain, 1);
     mbar_init(&c->q_empty, 1);
-    for (int i = 0; i < kNK; ++i) mbar_init(&c->k_empty[i], 1);
-    for (int i = 0; i < kNV; ++i) mbar_init(&c->v_empty[i], 1);
+    for (int i = 0; i < kN; ++i) mbar_init(&c->empty[i], 1);
     for (int i = 0; i < 2; ++i) mbar_init(&c->s_full[i], 1);
-    mbar_init(&c->o_done, 1);
+    for (int i = 0; i < 2; ++i) mbar_init(&c->o_done[i], 1);
     mbar_init(&c->v_fix, 1);
     mbar_init(&c->grp_sm, 128);
     c->abort_flag = 0;
@@ -171,8 +176,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
   Piece pc;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ Q + K slices
-    int kc = 0, pi = 0, q_issued = 0;
+    // ------------------------------------------------------------ producer: Q, then the ring in order
+    int sc = 0, pi = 0, q_issued = 0, fixc = 0;
     bool stop = false;
     while (!stop && it.next(pc)) {
       if (lane == 0) {
@@ -185,169 +190,173 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
           for (int j = 0; j < 9; ++j) tma_load_2d_pair(sQ + j * 8192, &tm_q, qbar, 64 * j, qy);
           ++q_issued;
         }
-        const int req = pc.unit;
-        const int npg = (p.seqlens[req] + kPage - 1) / kPage;
-        for (int k = pc.t0; k < pc.t1 && !stop; k += 2) {
-          // own tile; past the piece's end the pair's other tile is loaded again (its keys are masked)
+      }
+      stop = __shfl_sync(0xffffffffu, stop ? 1 : 0, 0) != 0;
+      const int req = pc.unit;
+      const int Ls = p.seqlens[req];
+      const int npg = (Ls + kPage - 1) / kPage;
+      const int nsteps = (pc.t1 - pc.t0 + 1) >> 1;
+      for (int h = 0; h <= 2 * nsteps && !stop; ++h) {
+        if (!ring_entry_exists(h, nsteps)) continue;
+        const int k = pc.t0 + 2 * ring_entry_step(h);
+        if (ring_entry_is_k(h)) {
+          // own tile; past the piece's end the pair's other tile is loaded
+          // again (its keys are masked)
           const int t = (k + (int)pr.rank < pc.t1) ? k + (int)pr.rank : k;
-          int pa = page_of(p, req, 2 * t, npg);
-          int pb = page_of(p, req, 2 * t + 1, npg);
-          if (pb < 0) pb = pa;
-          const int tp = t + 2 * kPrefetchSteps;
-          if (tp < pc.t1) {
-            for (int h = 0; h < 2; ++h) {
-              const int pf = page_of(p, req, 2 * tp + h, npg);
-              if (pf >= 0)
-                prefetch_l2(static_cast<const uint8_t*>(p.kcache) + (size_t)pf * kPage * kDqk * 2, kPage * kDqk * 2);
+          int pa = 0, pb = 0;
+          if (lane == 0) {
+            pa = page_of(p, req, 2 * t, npg);
+            pb = page_of(p, req, 2 * t + 1, npg);
+            if (pb < 0) pb = pa;
+            const int tp = t + 2 * kPrefetchSteps;
+            if (tp < pc.t1) {
+              for (int hh = 0; hh < 2; ++hh) {
+                const int pf = page_of(p, req, 2 * tp + hh, npg);
+                if (pf >= 0)
+                  prefetch_l2(static_cast<const uint8_t*>(p.kcache) + (size_t)pf * kPage * kDqk * 2,
+                              kPage * kDqk * 2);
+              }
             }
           }
-          for (int j = 0; j < 9; ++j, ++kc) {
-            const int slot = kc % kNK;
-            uint8_t* dst = sK + slot * kSlot;
-            if (!pwait(pr, &c->k_empty[slot], ((kc / kNK) & 1) ^ 1, p)) { stop = true; break; }
-            const uint32_t kbar = map_to_rank(smem_u32(&c->k_full[slot]), 0);
-            if (pr.leader) mbar_arrive_expect_tx(&c->k_full[slot], 2 * kSlot);
-            tma_load_2d_pair(dst, &tm_kv, kbar, 64 * j, pa * kPage);
-            tma_load_2d_pair(dst + 8192, &tm_kv, kbar, 64 * j, pb * kPage);
+          for (int j = 0; j < 9; ++j, ++sc) {
+            const int slot = sc % kN;
+            uint8_t* dst = sRing + slot * kSlot;
+            bool ok = true;
+            if (lane == 0) {
+              ok = pwait(pr, &c->empty[slot], ((sc / kN) & 1) ^ 1, p);
+              if (ok) {
+                const uint32_t bar = map_to_rank(smem_u32(&c->full[slot]), 0);
+                if (pr.leader) mbar_arrive_expect_tx(&c->full[slot], 2 * kSlot);
+                tma_load_2d_pair(dst, &tm_kv, bar, 64 * j, pa * kPage);
+                tma_load_2d_pair(dst + 8192, &tm_kv, bar, 64 * j, pb * kPage);
+              }
+            }
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok) { stop = true; break; }
+          }
+        } else {
+          // V: slot (q, jd) = page q of the step (tile k + q/2, page half
+          // q%2), value dims 256*jd + 128*rank + [0,128) as two 64-dim halves
+          for (int q = 0; q < 4 && !stop; ++q) {
+            const int tile = k + (q >> 1), pj = 2 * tile + (q & 1);
+            const int nv = tile < pc.t1 ? max(0, min(kPage, Ls - kPage * pj)) : 0;
+            int pg = 0;
+            if (lane == 0 && nv > 0) pg = page_of(p, req, pj, npg);
+            for (int jd = 0; jd < 2; ++jd, ++sc) {
+              const int slot = sc % kN;
+              uint8_t* dst = sRing + slot * kSlot;
+              bool ok = true;
+              if (lane == 0) ok = pwait(pr, &c->empty[slot], ((sc / kN) & 1) ^ 1, p);
+              ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+              if (!ok) { stop = true; break; }
+              const int x0 = 256 * jd + 128 * (int)pr.rank;
+              const uint32_t bar = map_to_rank(smem_u32(&c->full[slot]), 0);
+              // the even CTA expects both CTAs' bytes of every slot
+              if (lane == 0 && pr.leader) mbar_arrive_expect_tx(&c->full[slot], 2 * kSlot);
+              if (nv == kPage) {
+                if (lane == 0) {
+                  tma_load_2d_pair(dst, &tm_kv, bar, x0, pg * kPage);
+                  tma_load_2d_pair(dst + 8192, &tm_kv, bar, x0 + 64, pg * kPage);
+                }
+              } else {
+                // keys past the request's end have zero probability, but their
+                // cache rows may hold anything (0 x NaN = NaN): load locally,
+                // zero those rows, then report the slot's bytes as delivered
+                if (nv > 0) {
+                  if (lane == 0) {
+                    mbar_arrive_expect_tx(&c->v_fix, kSlot);
+                    tma_load_2d(dst, &tm_kv, &c->v_fix, x0, pg * kPage);
+                    tma_load_2d(dst + 8192, &tm_kv, &c->v_fix, x0 + 64, pg * kPage);
+                    ok = pwait(pr, &c->v_fix, fixc & 1, p);
+                  }
+                  ++fixc;
+                  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                  if (!ok) { stop = true; break; }
+                }
+                const uint4 z = make_uint4(0, 0, 0, 0);
+                for (int i = nv * 8 + lane; i < kPage * 8; i += 32) {  // 8 chunks of 16 B per 128-B row
+                  *reinterpret_cast<uint4*>(dst + i * 16) = z;
+                  *reinterpret_cast<uint4*>(dst + 8192 + i * 16) = z;
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                  fence_acq_rel_cluster();
+                  mbar_complete_tx_cluster(bar, kSlot);
+                }
+              }
+            }
           }
         }
       }
-      stop = __shfl_sync(0xffffffffu, stop ? 1 : 0, 0) != 0;
       ++pi;
     }
     if (lane == 0 && pr.leader) {  // the even CTA's barriers count both CTAs' copies
       if (q_issued > 0) mbar_wait_cluster(&c->q_full, (uint32_t)((q_issued - 1) & 1), p.timeout_ns);
-      for (int i = kc > kNK ? kc - kNK : 0; i < kc; ++i)
-        mbar_wait_cluster(&c->k_full[i % kNK], (uint32_t)((i / kNK) & 1), p.timeout_ns);
+      for (int i = sc > kN ? sc - kN : 0; i < sc; ++i)
+        mbar_wait_cluster(&c->full[i % kN], (uint32_t)((i / kN) & 1), p.timeout_ns);
     }
-    __syncwarp();
-  } else if (warp == 3) {
-    // ------------------------------------------------------------ V slots
-    // slot (q, jd): page q of the step (tile k + q/2, page half q%2), value
-    // dims 256*jd + 128*rank + [0,128) as two 64-dim halves.
-    int vc = 0, fixc = 0;
-    bool stop = false;
-    while (!stop && it.next(pc)) {
-      const int req = pc.unit;
-      const int Ls = p.seqlens[req];
-      const int npg = (Ls + kPage - 1) / kPage;
-      for (int k = pc.t0; k < pc.t1 && !stop; k += 2) {
-        for (int q = 0; q < 4 && !stop; ++q) {
-          const int tile = k + (q >> 1), pj = 2 * tile + (q & 1);
-          const int nv = tile < pc.t1 ? max(0, min(kPage, Ls - kPage * pj)) : 0;
-          const int pg = nv > 0 ? page_of(p, req, pj, npg) : 0;
-          for (int jd = 0; jd < 2; ++jd, ++vc) {
-            const int slot = vc % kNV;
-            uint8_t* dst = sV + slot * kSlot;
-            bool ok = true;
-            if (lane == 0) ok = pwait(pr, &c->v_empty[slot], ((vc / kNV) & 1) ^ 1, p);
-            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-            if (!ok) { stop = true; break; }
-            const int x0 = 256 * jd + 128 * (int)pr.rank;
-            if (nv == kPage) {
-              if (lane == 0) {
-                const uint32_t vbar = map_to_rank(smem_u32(&c->v_full[slot]), 0);
-                if (pr.leader) mbar_arrive_expect_tx(&c->v_full[slot], 2 * kSlot);
-                else mbar_arrive_cluster(vbar);
-                tma_load_2d_pair(dst, &tm_kv, vbar, x0, pg * kPage);
-                tma_load_2d_pair(dst + 8192, &tm_kv, vbar, x0 + 64, pg * kPage);
-              }
-            } else {
-              // keys past the request's end have zero probability, but their
-              // cache rows may hold anything (0 x NaN = NaN): load locally,
-              // zero those rows, then count the slot as full
-              if (nv > 0) {
-                if (lane == 0) {
-                  mbar_arrive_expect_tx(&c->v_fix, kSlot);
-                  tma_load_2d(dst, &tm_kv, &c->v_fix, x0, pg * kPage);
-                  tma_load_2d(dst + 8192, &tm_kv, &c->v_fix, x0 + 64, pg * kPage);
-                  ok = pwait(pr, &c->v_fix, fixc & 1, p);
-                }
-                ++fixc;
-                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-                if (!ok) { stop = true; break; }
-              }
-              const uint4 z = make_uint4(0, 0, 0, 0);
-              for (int i = nv * 8 + lane; i < kPage * 8; i += 32) {  // 8 chunks of 16 B per 128-B row
-                *reinterpret_cast<uint4*>(dst + i * 16) = z;
-                *reinterpret_cast<uint4*>(dst + 8192 + i * 16) = z;
-              }
-              fence_proxy_async_smem();
-              __syncwarp();
-              if (lane == 0) arrive_leader(pr, &c->v_full[slot]);
-            }
-          }
-        }
-      }
-    }
-    if (lane == 0 && pr.leader)
-      for (int i = vc > kNV ? vc - kNV : 0; i < vc; ++i)
-        mbar_wait_cluster(&c->v_full[i % kNV], (uint32_t)((i / kNV) & 1), p.timeout_ns);
     __syncwarp();
   } else if (warp == 1 && pr.leader) {
-    // ------------------------------------------------------------ S issuer
-    const uint32_t idesc = idesc_bf16(128, 256, false, false);
-    int kc = 0, gt = 0, pi = 0;
+    // ------------------------------------------------------------ MMA issuer: S(0), S(1), O(0), S(2), O(1), ...
+    const uint32_t idesc_s = idesc_bf16(128, 256, false, false);
+    const uint32_t idesc_o = idesc_bf16(128, 256, false, true);
+    int sc = 0, gs = 0, go = 0, pi = 0;
     bool stop = false;
     if (lane == 0) {
       while (!stop && it.next(pc)) {
         if (!pwait(pr, &c->q_full, pi & 1, p)) { stop = true; break; }
-        for (int k = pc.t0; k < pc.t1 && !stop; k += 2, ++gt) {
-          const int b = gt & 1;
-          if (!pwait(pr, &c->s_empty[b], ((gt >> 1) & 1) ^ 1, p)) { stop = true; break; }
-          tc_fence_after();
-          const uint32_t d = tmem + kTmemS + 128 * b;
-          for (int j = 0; j < 9; ++j, ++kc) {
-            const int slot = kc % kNK;
-            if (!pwait(pr, &c->k_full[slot], (kc / kNK) & 1, p)) { stop = true; break; }
+        const int nsteps = (pc.t1 - pc.t0 + 1) >> 1;
+        for (int h = 0; h <= 2 * nsteps && !stop; ++h) {
+          if (!ring_entry_exists(h, nsteps)) continue;
+          const int g = ring_entry_step(h);
+          if (ring_entry_is_k(h)) {
+            const int b = gs & 1;
+            if (!pwait(pr, &c->s_empty[b], ((gs >> 1) & 1) ^ 1, p)) { stop = true; break; }
             tc_fence_after();
-            const uint32_t qa = smem_u32(sQ + j * 8192), kb = smem_u32(sK + slot * kSlot);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_bf16_ss_pair(d, sdesc(qa + kk * 32, 16, 1024), sdesc(kb + kk * 32, 16, 1024), idesc,
-                               (j | kk) != 0 ? 1u : 0u);
-            mma_commit_pair(&c->k_empty[slot]);
-          }
-          if (!stop && !(gt == 0 && (p.debug_flags & MLA_DEBUG_WITHHOLD_SCORES))) mma_commit_pair(&c->s_full[b]);
-        }
-        if (!stop) mma_commit_pair(&c->q_empty);
-        ++pi;
-      }
-      mma_commit_pair(&c->drain_s);  // every MMA this thread issued has completed before teardown
-      mbar_wait(&c->drain_s, 0, p.timeout_ns);
-    }
-    __syncwarp();
-  } else if (warp == 2 && pr.leader) {
-    // ------------------------------------------------------------ O issuer
-    const uint32_t idesc = idesc_bf16(128, 256, false, true);
-    int vc = 0, gt = 0, pi = 0;
-    bool stop = false;
-    if (lane == 0) {
-      while (!stop && it.next(pc)) {
-        for (int k = pc.t0; k < pc.t1 && !stop; k += 2, ++gt) {
-          const bool first = (k == pc.t0);
-          if (first && pi > 0 && !pwait(pr, &c->o_free, (pi - 1) & 1, p)) { stop = true; break; }
-          if (!pwait(pr, &c->p_full, gt & 1, p)) { stop = true; break; }
-          const uint32_t pt = smem_u32(sP);
-          for (int q = 0; q < 4 && !stop; ++q) {
-            for (int jd = 0; jd < 2; ++jd, ++vc) {
-              const int slot = vc % kNV;
-              if (!pwait(pr, &c->v_full[slot], (vc / kNV) & 1, p)) { stop = true; break; }
+            const uint32_t d = tmem + kTmemS + 128 * b;
+            for (int j = 0; j < 9; ++j, ++sc) {
+              const int slot = sc % kN;
+              if (!pwait(pr, &c->full[slot], (sc / kN) & 1, p)) { stop = true; break; }
               tc_fence_after();
-              const uint32_t va = smem_u32(sV + slot * kSlot);
+              const uint32_t qa = smem_u32(sQ + j * 8192), kb = smem_u32(sRing + slot * kSlot);
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk)
-                mma_bf16_ss_pair(tmem + 128 * jd, sdesc(pt + q * 8192 + kk * 32, 16, 1024),
-                                 sdesc(va + kk * 2048, 8192, 1024), idesc, (first && q == 0 && kk == 0) ? 0u : 1u);
-              mma_commit_pair(&c->v_empty[slot]);
+                mma_bf16_ss_pair(d, sdesc(qa + kk * 32, 16, 1024), sdesc(kb + kk * 32, 16, 1024), idesc_s,
+                                 (j | kk) != 0 ? 1u : 0u);
+              mma_commit_pair(&c->empty[slot]);
             }
+            if (stop) break;
+            if (!(gs == 0 && (p.debug_flags & MLA_DEBUG_WITHHOLD_SCORES))) mma_commit_pair(&c->s_full[b]);
+            ++gs;
+            if (g == nsteps - 1) mma_commit_pair(&c->q_empty);  // Q is free once the last S completes
+          } else {
+            const bool first = g == 0;
+            if (first && pi > 0 && !pwait(pr, &c->o_free, (pi - 1) & 1, p)) { stop = true; break; }
+            if (!pwait(pr, &c->p_full[go & 1], (go >> 1) & 1, p)) { stop = true; break; }
+            const uint32_t pt = smem_u32(sP + (go & 1) * kPBytes);
+            for (int q = 0; q < 4 && !stop; ++q) {
+              for (int jd = 0; jd < 2; ++jd, ++sc) {
+                const int slot = sc % kN;
+                if (!pwait(pr, &c->full[slot], (sc / kN) & 1, p)) { stop = true; break; }
+                tc_fence_after();
+                const uint32_t va = smem_u32(sRing + slot * kSlot);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                  mma_bf16_ss_pair(tmem + 128 * jd, sdesc(pt + q * 8192 + kk * 32, 16, 1024),
+                                   sdesc(va + kk * 2048, 8192, 1024), idesc_o, (first && q == 0 && kk == 0) ? 0u : 1u);
+                mma_commit_pair(&c->empty[slot]);
+              }
+            }
+            if (stop) break;
+            mma_commit_pair(&c->o_done[go & 1]);
+            ++go;
           }
-          if (!stop) mma_commit_pair(&c->o_done);
         }
         ++pi;
       }
-      mma_commit_pair(&c->drain_o);
-      mbar_wait(&c->drain_o, 0, p.timeout_ns);
+      mma_commit_pair(&c->drain);  // every MMA this thread issued has completed before teardown
+      mbar_wait(&c->drain, 0, p.timeout_ns);
     }
     __syncwarp();
   } else if (warp >= 4) {
@@ -397,10 +406,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
           m_used = tmax;
           l_sum *= alpha;
         }
-        // pass 2: probabilities (masked by select) -> bf16 staged in TMEM over
-        // the S columns already read (keys 32w.. -> columns 16w..)
+        // P buffer b was last read by the O product of step gt - 2 (one
+        // barrier per buffer: O of step gt cannot complete before this
+        // thread's P, so the parity wait never falls two phases behind)
+        if (gt >= 2 && !pwait(pr, &c->o_done[b], ((gt >> 1) - 1) & 1, p)) { stop = true; break; }
+        // pass 2: probabilities (masked by select) -> bf16 -> P buffer b,
+        // K-major [64 rows][64 keys] per slice: keys 64s.. in slice s; this
+        // thread's keys are 128*half + [0,128), slices 2*half and 2*half + 1
         const float mc = (m_used == -INFINITY ? 0.f : m_used) * p.scale_log2;
         float part = 0.f;
+        uint8_t* pbuf = sP + b * kPBytes;
 #pragma unroll 1
         for (int w = 0; w < 4; ++w) {
           uint32_t sv[32];
@@ -417,15 +432,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
             pk[i] = pack_bf16x2(p0, p1);
             part += p0 + p1;
           }
-          tmem_st16(s_addr + 16 * w, pk);
+          uint8_t* rowp = pbuf + (2 * half + (w >> 1)) * 8192 + (row >> 3) * 1024 + (row & 7) * 128;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int ch = 4 * (w & 1) + q;
+            *reinterpret_cast<uint4*>(rowp + ((ch ^ (row & 7)) << 4)) =
+                make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+          }
         }
-        tmem_st_wait();
         l_sum += part;
-        // O MMAs of the previous step must be complete before O is rescaled
-        // and before P (which they read) is overwritten
-        if (gt >= 1 && !pwait(pr, &c->o_done, (gt - 1) & 1, p)) { stop = true; break; }
-        tc_fence_after();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) arrive_leader(pr, &c->s_empty[b]);  // this step's scores are consumed
         if (need) {
+          // O must hold every product up to step gt - 1 before it is rescaled
+          if (!pwait(pr, &c->o_done[(gt - 1) & 1], ((gt - 1) >> 1) & 1, p)) { stop = true; break; }
+          tc_fence_after();
 #pragma unroll 1
           for (int c16 = 0; c16 < 16; ++c16) {  // 2 x 128 columns of this row
             uint32_t ov[16];
@@ -438,28 +460,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
           }
           tmem_st_wait();
         }
-        // P, K-major [64 rows][64 keys] per slice: keys 64s.. in slice s; this
-        // thread's keys are 128*half + [0,128), slices 2*half and 2*half + 1
-#pragma unroll 1
-        for (int w = 0; w < 4; ++w) {
-          uint32_t pk[16];
-          tmem_ld16(s_addr + 16 * w, pk);
-          tmem_ld_wait();
-          uint8_t* rowp = sP + (2 * half + (w >> 1)) * 8192 + (row >> 3) * 1024 + (row & 7) * 128;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int ch = 4 * (w & 1) + q;
-            *reinterpret_cast<uint4*>(rowp + ((ch ^ (row & 7)) << 4)) =
-                make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-          }
-        }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) {
-          arrive_leader(pr, &c->s_empty[b]);  // scores and staged probabilities consumed
-          arrive_leader(pr, &c->p_full);
-        }
+        if (lane == 0) arrive_leader(pr, &c->p_full[b]);
         last_gt = gt;
       }
       if (stop) break;
@@ -467,7 +471,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
       c->lx[half][row] = l_sum;
       if (!group_sync(pr, gph, p)) { stop = true; break; }
       const float l_tot = l_sum + c->lx[half ^ 1][row];
-      if (last_gt >= 0 && !pwait(pr, &c->o_done, last_gt & 1, p)) { stop = true; break; }
+      if (last_gt >= 0 && !pwait(pr, &c->o_done[last_gt & 1], (last_gt >> 1) & 1, p)) { stop = true; break; }
       tc_fence_after();
       float inv = 0.f, lse = -INFINITY;
       if (l_tot > 0.f) {
@@ -531,7 +535,7 @@ cudaError_t launch_decode_pair(const CUtensorMap& tq, const CUtensorMap& tkv, co
   auto kern = pair::mla_decode_pair_kernel;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  kern<<<2 * parts, 256, smem, stream>>>(tq, tkv, p);
+  kern<<<2 * parts, pair::kThreads, smem, stream>>>(tq, tkv, p);
   return cudaGetLastError();
 }
 
@@ -541,7 +545,7 @@ int max_pair_clusters() {
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2, 1, 1);
-  cfg.blockDim = dim3(256, 1, 1);
+  cfg.blockDim = dim3(pair::kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cudaLaunchAttribute attr;
   attr.id = cudaLaunchAttributeClusterDimension;
