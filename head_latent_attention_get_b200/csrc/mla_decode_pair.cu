@@ -51,7 +51,6 @@ constexpr int kSlot = 16384;
 constexpr int kThreads = 256;
 constexpr int kQBytes = 9 * 8192;    // 64 rows x 576 dims
 constexpr int kPBytes = 4 * 8192;    // 64 rows x 256 tokens, per buffer
-constexpr int kPrefetchSteps = 2;    // L2 prefetch distance
 constexpr int kTmemCols = 512;
 constexpr int kTmemS = 256;          // S buffers at columns 256 and 384; O at 0 and 128
 constexpr float kRescaleLog2 = 8.0f;
@@ -68,7 +67,7 @@ struct Ctrl {
   // barriers counted on the even CTA (the MMA issuer) ...
   uint64_t q_full;                     // 1 arrival (+ both CTAs' Q bytes)
   uint64_t full[kN];                   // 1 arrival (+ both CTAs' bytes of the slot)
-  uint64_t s_empty[2], p_full[2], o_free;  // 8 arrivals: 4 softmax warps x 2 CTAs
+  uint64_t p_full[2], o_free;          // 8 arrivals: 4 softmax warps x 2 CTAs
   uint64_t drain;
   // ... and in each CTA
   uint64_t q_empty, empty[kN];         // pair-MMA commits
@@ -115,7 +114,8 @@ __device__ __forceinline__ bool group_sync(const Pair& pr, uint32_t& phase, cons
 
 // Arrive on barrier `bar` of the even CTA (a local arrive there, a remote one from the odd CTA).
 __device__ __forceinline__ void arrive_leader(const Pair& pr, uint64_t* bar) {
-  mbar_arrive_cluster(map_to_rank(smem_u32(bar), 0));
+  if (pr.leader) mbar_arrive(bar);
+  else mbar_arrive_cluster(map_to_rank(smem_u32(bar), 0));
 }
 
 // Ring order of a piece of n steps: h = 0 -> K of step 0; h = 2g+1 -> K of
@@ -123,6 +123,23 @@ __device__ __forceinline__ void arrive_leader(const Pair& pr, uint64_t* bar) {
 __device__ __forceinline__ bool ring_entry_exists(int h, int nsteps) { return !((h & 1) && (h >> 1) + 1 >= nsteps); }
 __device__ __forceinline__ bool ring_entry_is_k(int h) { return h == 0 || (h & 1); }
 __device__ __forceinline__ int ring_entry_step(int h) { return h == 0 ? 0 : (h & 1) ? (h >> 1) + 1 : (h >> 1) - 1; }
+
+// Page ids of a request for one warp: lane l holds the id of logical page
+// base + l, so a page is one shuffle away instead of a dependent global load.
+// Every call is made by all 32 lanes with the same arguments.
+struct PageWindow {
+  int base = -1 << 30, mine = -1;
+  __device__ __forceinline__ void cover(const DecodeParams& p, int req, int lo, int hi, int npg, int lane) {
+    if (lo < base || hi > base + 32) {
+      base = lo;
+      mine = page_of(p, req, base + lane, npg);
+    }
+  }
+  __device__ __forceinline__ int get(const DecodeParams& p, int req, int j, int npg, int lane) const {
+    const int v = __shfl_sync(0xffffffffu, mine, (j - base) & 31);
+    return (j >= base && j < base + 32) ? v : page_of(p, req, j, npg);
+  }
+};
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
@@ -146,7 +163,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(&c->q_full, 1);
     for (int i = 0; i < kN; ++i) mbar_init(&c->full[i], 1);
-    for (int i = 0; i < 2; ++i) { mbar_init(&c->s_empty[i], 8); mbar_init(&c->p_full[i], 8); }
+    for (int i = 0; i < 2; ++i) mbar_init(&c->p_full[i], 8);
     mbar_init(&c->o_free, 8);
     mbar_init(&c->drain, 1);
     mbar_init(&c->q_empty, 1);
@@ -196,6 +213,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int Ls = p.seqlens[req];
       const int npg = (Ls + kPage - 1) / kPage;
       const int nsteps = (pc.t1 - pc.t0 + 1) >> 1;
+      PageWindow pw;
       for (int h = 0; h <= 2 * nsteps && !stop; ++h) {
         if (!ring_entry_exists(h, nsteps)) continue;
         const int k = pc.t0 + 2 * ring_entry_step(h);
@@ -203,21 +221,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           // own tile; past the piece's end the pair's other tile is loaded
           // again (its keys are masked)
           const int t = (k + (int)pr.rank < pc.t1) ? k + (int)pr.rank : k;
-          int pa = 0, pb = 0;
-          if (lane == 0) {
-            pa = page_of(p, req, 2 * t, npg);
-            pb = page_of(p, req, 2 * t + 1, npg);
-            if (pb < 0) pb = pa;
-            const int tp = t + 2 * kPrefetchSteps;
-            if (tp < pc.t1) {
-              for (int hh = 0; hh < 2; ++hh) {
-                const int pf = page_of(p, req, 2 * tp + hh, npg);
-                if (pf >= 0)
-                  prefetch_l2(static_cast<const uint8_t*>(p.kcache) + (size_t)pf * kPage * kDqk * 2,
-                              kPage * kDqk * 2);
-              }
-            }
-          }
+          // pages of the previous step's V through the next steps' K (no L2
+          // prefetch: it would occupy this SM's TMA engine ahead of the loads)
+          pw.cover(p, req, max(0, 2 * k - 4), 2 * k + 8, npg, lane);
+          int pa = pw.get(p, req, 2 * t, npg, lane);
+          int pb = pw.get(p, req, 2 * t + 1, npg, lane);
+          if (pb < 0) pb = pa;
           for (int j = 0; j < 9; ++j, ++sc) {
             const int slot = sc % kN;
             uint8_t* dst = sRing + slot * kSlot;
@@ -240,8 +249,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           for (int q = 0; q < 4 && !stop; ++q) {
             const int tile = k + (q >> 1), pj = 2 * tile + (q & 1);
             const int nv = tile < pc.t1 ? max(0, min(kPage, Ls - kPage * pj)) : 0;
-            int pg = 0;
-            if (lane == 0 && nv > 0) pg = page_of(p, req, pj, npg);
+            const int pg = nv > 0 ? pw.get(p, req, pj, npg, lane) : 0;
             for (int jd = 0; jd < 2; ++jd, ++sc) {
               const int slot = sc % kN;
               uint8_t* dst = sRing + slot * kSlot;
@@ -311,8 +319,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           if (!ring_entry_exists(h, nsteps)) continue;
           const int g = ring_entry_step(h);
           if (ring_entry_is_k(h)) {
+            // S buffer b was last read by the softmax of step gs - 2, whose
+            // P the O product of step gs - 2 (issued just before) waited for
             const int b = gs & 1;
-            if (!pwait(pr, &c->s_empty[b], ((gs >> 1) & 1) ^ 1, p)) { stop = true; break; }
             tc_fence_after();
             const uint32_t d = tmem + kTmemS + 128 * b;
             for (int j = 0; j < 9; ++j, ++sc) {
@@ -441,9 +450,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
         }
         l_sum += part;
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) arrive_leader(pr, &c->s_empty[b]);  // this step's scores are consumed
         if (need) {
           // O must hold every product up to step gt - 1 before it is rescaled
           if (!pwait(pr, &c->o_done[(gt - 1) & 1], ((gt - 1) >> 1) & 1, p)) { stop = true; break; }
@@ -463,7 +469,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) arrive_leader(pr, &c->p_full[b]);
+        if (lane == 0) arrive_leader(pr, &c->p_full[b]);  // P written, O rescaled, scores consumed
         last_gt = gt;
       }
       if (stop) break;
