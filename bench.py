@@ -58,6 +58,14 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
+def decode_kernel_name(w, rows: int) -> str:
+    """The decode kernel the library launches for this workload: CTA pairs for
+    units of 65-128 rows on the BF16 paged cache, one CTA per row group otherwise."""
+    if w.kv == "bf16" and not w.topk and rows > 64:
+        return "mla_decode_pair_kernel"
+    return "mla_decode_kernel"
+
+
 def recorded_traffic(workload: str):
     """DRAM bytes per decode launch from the committed ncu summary, if it was
     taken on the current kernel sources; else None."""
@@ -347,7 +355,7 @@ def run_gpu(args):
             "traffic": traffic,
             "peak_source": f"{peak_src} (MEASURED_PEAKS.json burst figures)" if peak_src == "measured"
             else "fallback",
-            "kernel": "mla_decode_kernel",
+            "kernel": decode_kernel_name(w, runner.rows),
             "kernel_ms": dec_avg,
             "hbm_frac": achieved_gbs / hbm_peak, "tensor_frac": achieved_tf / tc_peak,
             "roofline_frac": max(t_hbm, t_tc) / (dec_avg * 1e-3),

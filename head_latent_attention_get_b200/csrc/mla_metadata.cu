@@ -11,6 +11,11 @@
 // C_u + overhead + k, so it belongs to part floor(position / payload): every
 // tile lands in exactly one part, parts are contiguous in (unit, tile)
 // order, and the number of parts touching unit u follows in closed form.
+// A piece of a split unit costs more than the fixed overhead suggests (its
+// partial result is written in fp32 and merged by the combine pass, and the
+// pipeline refills), so when the largest unit costs at most kSplitPenalty
+// tiles more than an even share, the payload is raised to that unit's cost:
+// equal units then map one to a part and are never split.
 // The cost axis is int32 (the prefix is stored in num_splits), so the sum of
 // all tile counts plus overheads must stay below 2^31.
 #include <cuda_runtime.h>
@@ -39,6 +44,14 @@ __host__ __device__ inline int2 cost_to_tile(const int32_t* C, int U, int total,
   return make_int2(lo, local > 0 ? (int)local : 0);
 }
 
+constexpr int kSplitPenalty = 8;  // tiles
+
+__host__ __device__ inline int choose_payload(int total, int parts, int max_cost) {
+  if (total <= 0) return 1;
+  const int even = (total + parts - 1) / parts;
+  return (max_cost > even && max_cost <= even + kSplitPenalty) ? max_cost : even;
+}
+
 __host__ __device__ inline int first_part_of(int Cu, int payload) {
   return (int)((Cu + kSchedOverhead) / payload);
 }
@@ -54,14 +67,16 @@ extern "C" mla_status_t mla_get_metadata_host(const int32_t* cache_seqlens, int 
   if (h_kv != 1) return MLA_ERR_UNSUPPORTED;
   const int U = topk > 0 ? batch * s_q : batch;
   // cost prefix C[0..U] kept in num_splits first, then replaced by split pointers
-  int total = 0;
+  int total = 0, max_cost = 0;
   for (int u = 0; u < U; ++u) {
     num_splits[u] = (int32_t)total;
     int n = unit_tiles(cache_seqlens, u, topk);
-    total += n > 0 ? n + kSchedOverhead : 0;
+    const int cost = n > 0 ? n + kSchedOverhead : 0;
+    total += cost;
+    max_cost = cost > max_cost ? cost : max_cost;
   }
   num_splits[U] = (int32_t)total;
-  const int payload = total > 0 ? (total + num_sm_parts - 1) / num_sm_parts : 1;
+  const int payload = choose_payload(total, num_sm_parts, max_cost);
   for (int p = 0; p < num_sm_parts; ++p) {
     const int2 b = cost_to_tile(num_splits, U, total, p * payload);
     const int2 e = cost_to_tile(num_splits, U, total, (p + 1) * payload);
@@ -118,6 +133,20 @@ __device__ int2 block_exclusive_scan(int v) {
   return make_int2(before, total);
 }
 
+__device__ int block_max(int v) {
+  __shared__ int warp_max[kMetaThreads / 32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
+  if (lane == 0) warp_max[warp] = v;
+  __syncthreads();
+  int m = 0;
+#pragma unroll
+  for (int i = 0; i < kMetaThreads / 32; ++i) m = max(m, warp_max[i]);
+  __syncthreads();
+  return m;
+}
+
 __global__ void __launch_bounds__(kMetaThreads) mla_metadata_kernel(const int32_t* __restrict__ seqlens,
                                                                    int U, int topk, int parts,
                                                                    int32_t* __restrict__ tile_md,
@@ -127,11 +156,14 @@ __global__ void __launch_bounds__(kMetaThreads) mla_metadata_kernel(const int32_
   const int per = (U + kMetaThreads - 1) / kMetaThreads;
   const int u0 = min(U, t * per), u1 = min(U, u0 + per);
   // 1. cost prefix C[u] -> num_splits[u], total -> num_splits[U]
-  int my = 0;
+  int my = 0, my_max = 0;
   for (int u = u0; u < u1; ++u) {
     int n = unit_tiles(seqlens, u, topk);
-    my += n > 0 ? n + kSchedOverhead : 0;
+    const int cost = n > 0 ? n + kSchedOverhead : 0;
+    my += cost;
+    my_max = max(my_max, cost);
   }
+  const int max_cost = block_max(my_max);
   const int2 sc = block_exclusive_scan(my);
   const int total = sc.y;
   int c = sc.x;
@@ -142,7 +174,7 @@ __global__ void __launch_bounds__(kMetaThreads) mla_metadata_kernel(const int32_
   }
   if (t == 0) {
     num_splits[U] = total;
-    s_payload = total > 0 ? (total + parts - 1) / parts : 1;
+    s_payload = choose_payload(total, parts, max_cost);
   }
   __syncthreads();
   const int payload = s_payload;

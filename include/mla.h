@@ -118,10 +118,12 @@ mla_status_t mla_get_num_sm_parts(int device, int s_q, int h_q, int h_kv, int to
  * ceil(cache_seqlens[b]/128) blocks of 128 tokens (two pages); sparse
  * decoding (topk > 0) has one unit per (b, i), i < s_q, with ceil(topk/128)
  * blocks of 128 index slots. Every unit costs its blocks plus a fixed
- * overhead of 3 blocks; the units are laid end to end and cut into
- * num_sm_parts ranges of equal cost, so one part covers a contiguous run of
- * (unit, block) pairs and a unit may be split across parts. The total cost
- * must stay below 2^31.
+ * overhead of 3 blocks; the units are laid end to end and cut into ranges of
+ * equal cost, so one part covers a contiguous run of (unit, block) pairs and
+ * a unit may be split across parts. The range length is
+ * ceil(total / num_sm_parts), raised to the largest unit's cost when that is
+ * at most 8 blocks more (equal units then take one part each and are not
+ * split; the trailing parts get no work). The total cost must stay below 2^31.
  *
  *   cache_seqlens  device int32 [batch]; read only when topk == 0 (may be
  *                  NULL when topk > 0).

@@ -10,6 +10,7 @@ import numpy as np
 
 TILE = 128
 OVERHEAD = 3
+SPLIT_PENALTY = 8
 
 
 def unit_tiles(seqlens, batch, s_q, topk):
@@ -65,6 +66,12 @@ def check_schedule(tile_md, num_splits, seqlens, batch, s_q, topk, parts):
                 assert ws == ptr[u] + j, (u, p, ws, ptr[u] + j)
     assert ptr[U] <= U + parts
     total = sum(x + OVERHEAD for x in n if x > 0)
-    payload = -(-total // parts) if total else 1
+    even = -(-total // parts) if total else 1
+    unit_max = max([x + OVERHEAD for x in n if x > 0], default=0)
+    # the range grows to the largest unit's cost when that is at most
+    # SPLIT_PENALTY tiles above an even share (no split of equal units)
+    payload = unit_max if even < unit_max <= even + SPLIT_PENALTY else even
     assert max(cost) <= payload + 2 * OVERHEAD, (max(cost), payload)
+    if payload == unit_max and len(set(x for x in n if x > 0)) == 1:
+        assert ptr[U] == sum(1 for x in n if x > 0), "equal units must not be split"
     return {"payload": payload, "max_cost": max(cost), "splits": int(ptr[U])}
