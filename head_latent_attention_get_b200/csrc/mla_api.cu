@@ -83,8 +83,16 @@ mla_status_t run_decode(const mla_decode_args* a, const int32_t* indices, int to
   CUtensorMap tq, tkv;
   std::memset(&tkv, 0, sizeof(tkv));
   if (!make_map(&tq, a->q, (uint64_t)U * rows, kDqk, kDqk * 2, 64, 64)) return MLA_ERR_CUDA;
+  const int row_groups = (rows + kRowsPerCta - 1) / kRowsPerCta;
+  // more than 64 rows on the BF16 cache (paged or sparse): one CTA pair per
+  // part shares each cache tile between the two row halves
+  const bool pair = row_groups == 2 && mode != kModeFp8;
   if (mode == kModeBf16 &&
       !make_map(&tkv, a->kcache, (uint64_t)a->num_pages * kPage, kDqk, kDqk * 2, 64, 64))
+    return MLA_ERR_CUDA;
+  // sparse rows are gathered four at a time: boxes one row high
+  if (pair && mode == kModeSparse &&
+      !make_map(&tkv, a->kcache, (uint64_t)a->num_pages * kPage, kDqk, kDqk * 2, 64, 1))
     return MLA_ERR_CUDA;
   const WsLayout w = ws_layout(U, rows, a->num_sm_parts);
   char* ws = static_cast<char*>(a->workspace);
@@ -114,13 +122,9 @@ mla_status_t run_decode(const mla_decode_args* a, const int32_t* indices, int to
   p.status = reinterpret_cast<uint32_t*>(ws);
   p.timeout_ns = a->timeout_ns ? a->timeout_ns : 2000000000ull;
   p.debug_flags = a->debug_flags;
-  const int row_groups = (rows + kRowsPerCta - 1) / kRowsPerCta;
   const int rows_per_cta = rows < kRowsPerCta ? rows : kRowsPerCta;
-  // more than 64 rows on the BF16 paged cache: one CTA pair per part shares each
-  // cache tile between the two row halves instead of loading it twice
-  const cudaError_t e = (mode == kModeBf16 && row_groups == 2)
-                            ? launch_decode_pair(tq, tkv, p, a->num_sm_parts, stream)
-                            : launch_decode(rows_per_cta, mode, tq, tkv, p, a->num_sm_parts, row_groups, stream);
+  const cudaError_t e = pair ? launch_decode_pair(tq, tkv, p, a->num_sm_parts, mode == kModeSparse, stream)
+                             : launch_decode(rows_per_cta, mode, tq, tkv, p, a->num_sm_parts, row_groups, stream);
   if (e != cudaSuccess) return MLA_ERR_CUDA;
   if (a->debug_flags & MLA_DEBUG_SKIP_COMBINE) return MLA_OK;
   return launch_combine(a->workspace, U, rows, a->num_sm_parts, a->num_splits, a->out, a->lse, stream);

@@ -45,7 +45,6 @@ constexpr int kNK = 4;                 // K ring slots: 128 tokens x 64 dims (16
 constexpr int kNV = 4;                 // V ring slots: 64 tokens x 128 dims (16 KB)
 constexpr int kSlot = 16384;
 constexpr int kLag = 3;                // gather groups retire a slot 3 slots after issuing it
-constexpr int kPrefetchTiles = 3;      // L2 prefetch distance (bf16 paged)
 constexpr int kQBytes = 9 * 8192;      // 64 rows x 576 dims
 constexpr int kTmemCols = 512;
 constexpr int kTmemS = 256;            // S buffers at columns 256 and 384
@@ -320,14 +319,6 @@ __global__ void __launch_bounds__(MODE == kModeBf16 ? 256 : 320, 1)
             int pa = page_of(p, req, 2 * k, npg);
             int pb = page_of(p, req, 2 * k + 1, npg);
             if (pb < 0) pb = pa;  // half tile: reload page A, its keys are masked
-            if (rg == 0 && k + kPrefetchTiles < pc.t1) {  // warm L2 a few tiles ahead
-              for (int h = 0; h < 2; ++h) {
-                const int pf = page_of(p, req, 2 * (k + kPrefetchTiles) + h, npg);
-                if (pf >= 0)
-                  prefetch_l2(static_cast<const uint8_t*>(p.kcache) + (size_t)pf * kPage * kDqk * 2,
-                              kPage * kDqk * 2);
-              }
-            }
             for (int j = 0; j < 9; ++j, ++kc) {
               const int slot = kc % kNK;
               uint8_t* dst = sK + slot * kSlot;

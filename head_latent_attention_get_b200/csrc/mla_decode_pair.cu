@@ -1,5 +1,6 @@
-// MLA decode for units with more than 64 query rows (e.g. 128 heads), BF16
-// paged cache: one CTA pair (cluster of 2 CTAs on two SMs) per scheduler part.
+// MLA decode for units with more than 64 query rows (e.g. 128 heads) on the
+// BF16 cache, paged or token-sparse: one CTA pair (cluster of 2 CTAs on two
+// SMs) per scheduler part.
 //
 // Same computation as mla_decode.cu -- per unit, softmax(scale * Q K^T) V with
 // K = the 576-dim latent row and V = its first 512 dims ([flashinfer] ...
@@ -73,11 +74,13 @@ struct Ctrl {
   uint64_t q_empty, empty[kN];         // pair-MMA commits
   uint64_t s_full[2], o_done[2];       // pair-MMA commits; o_done[g & 1] completes O of step g
   uint64_t v_fix;                      // local loads of partial pages
+  uint64_t m_full[4];                  // sparse: key-validity mask of a step written (producer)
   uint64_t grp_sm;                     // 128 softmax threads
   uint32_t tmem_base;
   int abort_flag;
   float mx[2][2][64];                  // [step parity][token half][row]: per-half tile max
   float lx[2][64];                     // [token half][row]: per-half row sum
+  __align__(16) uint32_t vmask[4][8];  // sparse: [step % 4][tile half * 4 + word]: bit s = key 32*word + s valid
 };
 static_assert(sizeof(Ctrl) <= 2048, "control block");
 
@@ -141,6 +144,77 @@ struct PageWindow {
   }
 };
 
+// Sparse: resolves the 256 index slots of the step whose first tile is k.
+// Lane l ends with the cache rows of slots 4l..4l+3 of tile k in r[0..3] and
+// of tile k+1 in r[4..7]. Ignored slots (-1), out-of-range indices (also
+// reported in the status word), slots past topk and slots of tiles outside
+// the piece get a row past the end of the cache, which the gather zero-fills.
+// The step's key-validity bits go to mask[4*h + w], bit s = key 32w + s of
+// tile k + h.
+__device__ __forceinline__ void resolve_sparse_step(const DecodeParams& p, int unit, int b, int L, int k, int t1,
+                                                    int lane, int (&r)[8], uint32_t* mask) {
+  const int oob = p.num_pages * kPage;
+  int idx[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const int tile = k + (e >> 2);
+    const int slot = kTile * tile + 4 * lane + (e & 3);
+    idx[e] = (tile < t1 && slot < p.topk) ? p.indices[(size_t)unit * p.topk + slot] : -1;
+  }
+  int pg[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const bool in = idx[e] >= 0 && idx[e] < L;
+    const int j = in ? idx[e] / kPage : 0;
+    const bool jin = in && j < p.bt_stride;
+    if (idx[e] != -1 && !jin) atomicOr(p.status, (uint32_t)MLA_DEVICE_STATUS_BOUNDS);
+    pg[e] = jin ? p.block_table[(size_t)b * p.bt_stride + j] : -1;
+    if (!jin) idx[e] = -1;
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const bool ok = idx[e] >= 0 && pg[e] >= 0 && pg[e] < p.num_pages;
+    if (idx[e] >= 0 && !ok) atomicOr(p.status, (uint32_t)MLA_DEVICE_STATUS_BOUNDS);
+    r[e] = ok ? pg[e] * kPage + idx[e] % kPage : oob;
+  }
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t v = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v |= (r[4 * h + i] != oob ? 1u : 0u) << i;
+    v <<= 4 * (lane & 7);
+    v |= __shfl_xor_sync(0xffffffffu, v, 1);
+    v |= __shfl_xor_sync(0xffffffffu, v, 2);
+    v |= __shfl_xor_sync(0xffffffffu, v, 4);
+    if ((lane & 7) == 0) mask[4 * h + (lane >> 3)] = v;
+  }
+}
+
+// Sparse: the K slice j of this CTA's tile (lane l gathers rows 4l..4l+3).
+__device__ __forceinline__ void gather_k_slice(uint8_t* dst, const CUtensorMap* map, uint32_t bar, int j, int lane,
+                                               const int (&r)[8], uint32_t rank) {
+  const int a = rank ? r[4] : r[0], b = rank ? r[5] : r[1], c = rank ? r[6] : r[2], d = rank ? r[7] : r[3];
+  tma_gather4_pair(dst + 4 * lane * 128, map, bar, 64 * j, a, b, c, d);
+}
+
+// Sparse: the V slot (q, jd): keys 64q..64q+63 of the step, value dims
+// 256*jd + 128*rank + [0,128) as two 64-dim halves; lanes 16(q%2)..16(q%2)+15
+// hold the rows.
+template <int Q>
+__device__ __forceinline__ void gather_v_slot(uint8_t* dst, const CUtensorMap* map, uint32_t bar, int jd, int lane,
+                                              const int (&r)[8], uint32_t rank) {
+  const int l0 = 16 * (Q & 1);
+  if (lane >= l0 && lane < l0 + 16) {
+    const int e = 4 * (Q >> 1);
+    uint8_t* row = dst + (4 * (lane - l0)) * 128;
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh)
+      tma_gather4_pair(row + hh * 8192, map, bar, 256 * jd + 128 * (int)rank + 64 * hh, r[e], r[e + 1], r[e + 2],
+                       r[e + 3]);
+  }
+}
+
+template <bool SPARSE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
                            const DecodeParams p) {
@@ -171,6 +245,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) mbar_init(&c->s_full[i], 1);
     for (int i = 0; i < 2; ++i) mbar_init(&c->o_done[i], 1);
     mbar_init(&c->v_fix, 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&c->m_full[i], 1);
     mbar_init(&c->grp_sm, 128);
     c->abort_flag = 0;
     fence_mbar_init();
@@ -195,6 +270,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer: Q, then the ring in order
     int sc = 0, pi = 0, q_issued = 0, fixc = 0;
+    int gk = 0, gv = 0;        // steps whose K / V this warp has issued (all pieces)
+    int rs0[8], rs1[8];        // sparse: cache rows of steps with even / odd gk
     bool stop = false;
     while (!stop && it.next(pc)) {
       if (lane == 0) {
@@ -209,7 +286,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
       }
       stop = __shfl_sync(0xffffffffu, stop ? 1 : 0, 0) != 0;
-      const int req = pc.unit;
+      const int req = unit_req(p, pc.unit);
       const int Ls = p.seqlens[req];
       const int npg = (Ls + kPage - 1) / kPage;
       const int nsteps = (pc.t1 - pc.t0 + 1) >> 1;
@@ -217,7 +294,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       for (int h = 0; h <= 2 * nsteps && !stop; ++h) {
         if (!ring_entry_exists(h, nsteps)) continue;
         const int k = pc.t0 + 2 * ring_entry_step(h);
-        if (ring_entry_is_k(h)) {
+        if (ring_entry_is_k(h) && SPARSE) {
+          if (gk & 1) resolve_sparse_step(p, pc.unit, req, Ls, k, pc.t1, lane, rs1, c->vmask[gk & 3]);
+          else resolve_sparse_step(p, pc.unit, req, Ls, k, pc.t1, lane, rs0, c->vmask[gk & 3]);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&c->m_full[gk & 3]);  // the softmax of this step reads the mask
+          for (int j = 0; j < 9; ++j, ++sc) {
+            const int slot = sc % kN;
+            bool ok = true;
+            if (lane == 0) ok = pwait(pr, &c->empty[slot], ((sc / kN) & 1) ^ 1, p);
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok) { stop = true; break; }
+            const uint32_t bar = map_to_rank(smem_u32(&c->full[slot]), 0);
+            if (lane == 0 && pr.leader) mbar_arrive_expect_tx(&c->full[slot], 2 * kSlot);
+            __syncwarp();
+            if (gk & 1) gather_k_slice(sRing + slot * kSlot, &tm_kv, bar, j, lane, rs1, pr.rank);
+            else gather_k_slice(sRing + slot * kSlot, &tm_kv, bar, j, lane, rs0, pr.rank);
+          }
+          ++gk;
+        } else if (ring_entry_is_k(h)) {
           // own tile; past the piece's end the pair's other tile is loaded
           // again (its keys are masked)
           const int t = (k + (int)pr.rank < pc.t1) ? k + (int)pr.rank : k;
@@ -227,6 +322,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           int pa = pw.get(p, req, 2 * t, npg, lane);
           int pb = pw.get(p, req, 2 * t + 1, npg, lane);
           if (pb < 0) pb = pa;
+          ++gk;
           for (int j = 0; j < 9; ++j, ++sc) {
             const int slot = sc % kN;
             uint8_t* dst = sRing + slot * kSlot;
@@ -243,6 +339,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
             if (!ok) { stop = true; break; }
           }
+        } else if (SPARSE) {
+          // V of the step: slot (q, jd) = keys 64q..64q+63, value dims
+          // 256*jd + 128*rank + [0,128) as two 64-dim halves
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+#pragma unroll
+            for (int jd = 0; jd < 2; ++jd) {
+              const int slot = sc % kN;
+              bool ok = !stop;
+              if (lane == 0 && ok) ok = pwait(pr, &c->empty[slot], ((sc / kN) & 1) ^ 1, p);
+              ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+              if (!ok) { stop = true; continue; }
+              const uint32_t bar = map_to_rank(smem_u32(&c->full[slot]), 0);
+              if (lane == 0 && pr.leader) mbar_arrive_expect_tx(&c->full[slot], 2 * kSlot);
+              __syncwarp();
+              uint8_t* dst = sRing + slot * kSlot;
+              if (gv & 1) {
+                if (q == 0) gather_v_slot<0>(dst, &tm_kv, bar, jd, lane, rs1, pr.rank);
+                if (q == 1) gather_v_slot<1>(dst, &tm_kv, bar, jd, lane, rs1, pr.rank);
+                if (q == 2) gather_v_slot<2>(dst, &tm_kv, bar, jd, lane, rs1, pr.rank);
+                if (q == 3) gather_v_slot<3>(dst, &tm_kv, bar, jd, lane, rs1, pr.rank);
+              } else {
+                if (q == 0) gather_v_slot<0>(dst, &tm_kv, bar, jd, lane, rs0, pr.rank);
+                if (q == 1) gather_v_slot<1>(dst, &tm_kv, bar, jd, lane, rs0, pr.rank);
+                if (q == 2) gather_v_slot<2>(dst, &tm_kv, bar, jd, lane, rs0, pr.rank);
+                if (q == 3) gather_v_slot<3>(dst, &tm_kv, bar, jd, lane, rs0, pr.rank);
+              }
+              ++sc;
+            }
+          }
+          ++gv;
         } else {
           // V: slot (q, jd) = page q of the step (tile k + q/2, page half
           // q%2), value dims 256*jd + 128*rank + [0,128) as two 64-dim halves
@@ -380,15 +507,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     int gt = 0;
     bool stop = false;
     while (!stop && it.next(pc)) {
-      const int req = pc.unit;
+      const int req = unit_req(p, pc.unit);
       const int Ls = p.seqlens[req];
       const int limit = p.causal ? Ls - p.s_q + grow / p.h_q + 1 : Ls;
       float m_used = -INFINITY, l_sum = 0.f;
       int last_gt = -1;
       for (int k = pc.t0; k < pc.t1 && !stop; k += 2, ++gt) {
         const int b = gt & 1;
-        const int tile = k + half;
-        const int nv = (rvalid && tile < pc.t1) ? dense_tile_valid(limit, tile) : 0;
+        // validity of this thread's 128 keys: bit i of word w = key 32w + i
+        uint4 vm;
+        if (SPARSE) {
+          if (!pwait(pr, &c->m_full[gt & 3], (gt >> 2) & 1, p)) { stop = true; break; }
+          vm = rvalid ? *reinterpret_cast<const uint4*>(&c->vmask[gt & 3][4 * half]) : make_uint4(0, 0, 0, 0);
+        } else {
+          const int tile = k + half;
+          const int nv = (rvalid && tile < pc.t1) ? dense_tile_valid(limit, tile) : 0;
+          auto word = [nv](int w) {
+            const int nb = min(32, max(0, nv - 32 * w));
+            return nb >= 32 ? 0xffffffffu : ((1u << nb) - 1u);
+          };
+          vm = make_uint4(word(0), word(1), word(2), word(3));
+        }
         if (!pwait(pr, &c->s_full[b], (gt >> 1) & 1, p)) { stop = true; break; }
         tc_fence_after();
         const uint32_t s_addr = tmem + lane_base + kTmemS + 128 * b;
@@ -399,9 +538,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           uint32_t sv[32];
           tmem_ld32(s_addr + 32 * w, sv);
           tmem_ld_wait();
-          const int nb = min(32, max(0, nv - 32 * w));
+          const uint32_t mw = pick4u(vm, w);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) tmax = fmaxf(tmax, i < nb ? __uint_as_float(sv[i]) : -INFINITY);
+          for (int i = 0; i < 32; ++i) tmax = fmaxf(tmax, ((mw >> i) & 1u) ? __uint_as_float(sv[i]) : -INFINITY);
         }
         c->mx[gt & 1][half][row] = tmax;
         if (!group_sync(pr, gph, p)) { stop = true; break; }
@@ -430,14 +569,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           uint32_t sv[32];
           tmem_ld32(s_addr + 32 * w, sv);
           tmem_ld_wait();
-          const int nb = min(32, max(0, nv - 32 * w));
+          const uint32_t mw = pick4u(vm, w);
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const float e0 = ex2_approx(fmaf(__uint_as_float(sv[2 * i]), p.scale_log2, -mc));
             const float e1 = ex2_approx(fmaf(__uint_as_float(sv[2 * i + 1]), p.scale_log2, -mc));
-            const float p0 = (2 * i < nb) ? e0 : 0.f;
-            const float p1 = (2 * i + 1 < nb) ? e1 : 0.f;
+            const float p0 = ((mw >> (2 * i)) & 1u) ? e0 : 0.f;
+            const float p1 = ((mw >> (2 * i + 1)) & 1u) ? e1 : 0.f;
             pk[i] = pack_bf16x2(p0, p1);
             part += p0 + p1;
           }
@@ -536,9 +675,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 }  // namespace pair
 
 cudaError_t launch_decode_pair(const CUtensorMap& tq, const CUtensorMap& tkv, const DecodeParams& p, int parts,
-                               cudaStream_t stream) {
+                               bool sparse, cudaStream_t stream) {
   constexpr int smem = pair::Smem::total + 1024;
-  auto kern = pair::mla_decode_pair_kernel;
+  auto kern = sparse ? pair::mla_decode_pair_kernel<true> : pair::mla_decode_pair_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   kern<<<2 * parts, pair::kThreads, smem, stream>>>(tq, tkv, p);
@@ -547,7 +686,7 @@ cudaError_t launch_decode_pair(const CUtensorMap& tq, const CUtensorMap& tkv, co
 
 int max_pair_clusters() {
   constexpr int smem = pair::Smem::total + 1024;
-  auto kern = pair::mla_decode_pair_kernel;
+  auto kern = pair::mla_decode_pair_kernel<false>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2, 1, 1);

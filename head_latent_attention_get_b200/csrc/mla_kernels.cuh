@@ -31,9 +31,10 @@ struct DecodeParams {
 
 cudaError_t launch_decode(int rows_per_cta, int mode, const CUtensorMap& tq, const CUtensorMap& tkv,
                           const DecodeParams& p, int parts, int row_groups, cudaStream_t stream);
-// Units of more than 64 rows, BF16 paged cache: CTA pairs (clusters of two), one per part.
+// Units of more than 64 rows, BF16 cache (paged, or token-sparse when `sparse`):
+// CTA pairs (clusters of two), one per part.
 cudaError_t launch_decode_pair(const CUtensorMap& tq, const CUtensorMap& tkv, const DecodeParams& p, int parts,
-                               cudaStream_t stream);
+                               bool sparse, cudaStream_t stream);
 // How many CTA pairs of the pair kernel can be resident at once on the current device (0 if unknown).
 int max_pair_clusters();
 mla_status_t launch_metadata(const int32_t* seqlens, int U, int topk, int parts, int32_t* tile_md,

@@ -29,7 +29,9 @@ def _run(inp, **kw):
     ([300, 1000], 1, 16, 128),
     ([300, 1000], 1, 64, 192),          # last 128-slot tile is half full
     ([4000, 129, 2000], 2, 32, 256),    # s_q = 2: one unit per (request, query token)
-    ([5000, 3000], 1, 128, 512),        # two row groups
+    ([5000, 3000], 1, 128, 512),        # 128 rows: CTA pairs
+    ([300, 1000, 70], 1, 128, 192),     # CTA pairs, half-full last tile, odd tile count
+    ([4000, 129], 2, 96, 256),          # CTA pairs with 32 rows in the odd CTA, s_q = 2
 ])
 def test_sparse_vs_oracle(seqlens, s_q, h_q, topk):
     inp = _sparse(len(seqlens), seqlens, s_q, h_q, topk, seed=sum(seqlens) + topk)
@@ -39,8 +41,9 @@ def test_sparse_vs_oracle(seqlens, s_q, h_q, topk):
     assert r.status()[0] == C.MLA_OK
 
 
-def test_sparse_duplicates_and_all_ignored_rows():
-    inp = _sparse(2, [700, 700], 1, 32, 128, neg_frac=0.0, seed=9)
+@pytest.mark.parametrize("h_q", [32, 128])  # 128 rows run on CTA pairs
+def test_sparse_duplicates_and_all_ignored_rows(h_q):
+    inp = _sparse(2, [700, 700], 1, h_q, 128, neg_frac=0.0, seed=9)
     idx = inp.indices
     idx[0, 0, 64:] = idx[0, 0, :64]        # every key of request 0 counted twice
     idx[1, 0, :] = -1                      # request 1: empty key set -> out 0, lse -inf
@@ -51,8 +54,9 @@ def test_sparse_duplicates_and_all_ignored_rows():
     assert r.status()[0] == C.MLA_OK
 
 
-def test_out_of_range_indices_are_ignored_and_reported():
-    inp = _sparse(2, [500, 300], 1, 16, 128, seed=3)
+@pytest.mark.parametrize("h_q", [16, 128])
+def test_out_of_range_indices_are_ignored_and_reported(h_q):
+    inp = _sparse(2, [500, 300], 1, h_q, 128, seed=3)
     inp.indices[0, 0, 5] = 500             # == seqlen: out of range
     inp.indices[1, 0, 7] = -5              # negative but not -1
     out, lse, r = _run(inp)
@@ -62,10 +66,11 @@ def test_out_of_range_indices_are_ignored_and_reported():
     G.compare(out, lse, ref_o, ref_l, "out-of-range ignored")
 
 
-def test_ignored_slots_are_bit_exact():
+@pytest.mark.parametrize("h_q", [64, 128])
+def test_ignored_slots_are_bit_exact(h_q):
     """(i) NaN in every cache row that no valid index reaches changes no bit;
     (ii) appending a tile of -1 slots changes no bit."""
-    inp = _sparse(2, [900, 2000], 1, 64, 256, neg_frac=0.1, seed=21)
+    inp = _sparse(2, [900, 2000], 1, h_q, 256, neg_frac=0.1, seed=21)
     base_o, base_l, _ = _run(inp, num_sm_parts=2)
     # (i) poison all unreferenced tokens of both requests
     pois = dataclasses.replace(inp, kcache=inp.kcache.clone())
@@ -87,8 +92,9 @@ def test_ignored_slots_are_bit_exact():
     assert np.array_equal(el.view(np.uint32), one_l.view(np.uint32))
 
 
-def test_all_positions_in_order_equal_dense():
-    w = dataclasses.replace(W.get_workload("tiny"), batch=2, seqlens=[300, 190], h_q=64, seed=5)
+@pytest.mark.parametrize("h_q", [64, 128])
+def test_all_positions_in_order_equal_dense(h_q):
+    w = dataclasses.replace(W.get_workload("tiny"), batch=2, seqlens=[300, 190], h_q=h_q, seed=5)
     dense = W.make_inputs(w)
     idx = torch.full((2, 1, 320), -1, dtype=torch.int32)
     for b, L in enumerate([300, 190]):
