@@ -90,10 +90,6 @@ mla_status_t run_decode(const mla_decode_args* a, const int32_t* indices, int to
   if (mode == kModeBf16 &&
       !make_map(&tkv, a->kcache, (uint64_t)a->num_pages * kPage, kDqk, kDqk * 2, 64, 64))
     return MLA_ERR_CUDA;
-  // sparse rows are gathered four at a time: boxes one row high
-  if (pair && mode == kModeSparse &&
-      !make_map(&tkv, a->kcache, (uint64_t)a->num_pages * kPage, kDqk, kDqk * 2, 64, 1))
-    return MLA_ERR_CUDA;
   const WsLayout w = ws_layout(U, rows, a->num_sm_parts);
   char* ws = static_cast<char*>(a->workspace);
   DecodeParams p;

@@ -31,9 +31,13 @@
 // look-ahead. The MMA issuer follows the same order: S(0), S(1), O(0), S(2),
 // O(1), ...
 //
-// Warp roles (256 threads per CTA):
-//   0 Q, K and V via TMA (both CTAs; completion counted on the even CTA's barriers)
-//   1 TMEM allocation (both) and MMA issue (even CTA)
+// Warp roles (256 threads per CTA; 320 with sparse indices):
+//   0 Q (and, paged, K and V) via TMA (both CTAs; completion counted on the
+//     even CTA's barriers)
+//   1 TMEM allocation (both) and MMA issue (even CTA); sparse: forwarding of
+//     the odd CTA's slot completions (odd CTA)
+//   2, 3, 8, 9 sparse: row gathers with cp.async (both CTAs); a TMA row gather
+//     moves only ~7 B/clk per SM, cp.async from four warps about 20
 //   4-7 softmax + epilogue (both): thread i = (row i % 64, token half i / 64)
 // All waits are bounded; a timeout sets MLA_DEVICE_STATUS_TIMEOUT, raises the
 // abort flag of both CTAs, and every role winds down to the final cluster
@@ -49,7 +53,8 @@ namespace pair {
 constexpr int kN = 5;                // ring slots of 16 KB: a K slice (128 tokens x 64 dims)
                                      // or a V slot (64 tokens x 128 value dims, two 8 KB halves)
 constexpr int kSlot = 16384;
-constexpr int kThreads = 256;
+constexpr int kThreads = 256;         // paged
+constexpr int kThreadsSparse = 320;   // + four cp.async loader warps (2, 3, 8, 9)
 constexpr int kQBytes = 9 * 8192;    // 64 rows x 576 dims
 constexpr int kPBytes = 4 * 8192;    // 64 rows x 256 tokens, per buffer
 constexpr int kTmemCols = 512;
@@ -74,7 +79,8 @@ struct Ctrl {
   uint64_t q_empty, empty[kN];         // pair-MMA commits
   uint64_t s_full[2], o_done[2];       // pair-MMA commits; o_done[g & 1] completes O of step g
   uint64_t v_fix;                      // local loads of partial pages
-  uint64_t m_full[4];                  // sparse: key-validity mask of a step written (producer)
+  uint64_t m_full[4];                  // sparse: key-validity mask of a step written (4 loader warps)
+  uint64_t v_loc[kN];                  // sparse, odd CTA: its 128 loader threads
   uint64_t grp_sm;                     // 128 softmax threads
   uint32_t tmem_base;
   int abort_flag;
@@ -144,78 +150,29 @@ struct PageWindow {
   }
 };
 
-// Sparse: resolves the 256 index slots of the step whose first tile is k.
-// Lane l ends with the cache rows of slots 4l..4l+3 of tile k in r[0..3] and
-// of tile k+1 in r[4..7]. Ignored slots (-1), out-of-range indices (also
-// reported in the status word), slots past topk and slots of tiles outside
-// the piece get a row past the end of the cache, which the gather zero-fills.
-// The step's key-validity bits go to mask[4*h + w], bit s = key 32w + s of
-// tile k + h.
-__device__ __forceinline__ void resolve_sparse_step(const DecodeParams& p, int unit, int b, int L, int k, int t1,
-                                                    int lane, int (&r)[8], uint32_t* mask) {
-  const int oob = p.num_pages * kPage;
-  int idx[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    const int tile = k + (e >> 2);
-    const int slot = kTile * tile + 4 * lane + (e & 3);
-    idx[e] = (tile < t1 && slot < p.topk) ? p.indices[(size_t)unit * p.topk + slot] : -1;
+// Sparse: cache row of index slot `slot` of unit `unit` (request b, whose
+// cache holds L tokens), or -1 when the slot is ignored: -1 entries (silently),
+// out-of-range indices and page ids (reported in the status word), slots past
+// topk and slots of tiles outside the piece [.., t1).
+__device__ __forceinline__ int sparse_slot_row(const DecodeParams& p, int unit, int b, int L, int slot, int t1) {
+  if (slot / kTile >= t1 || slot >= p.topk) return -1;
+  const int idx = p.indices[(size_t)unit * p.topk + slot];
+  if (idx == -1) return -1;
+  const int j = idx / kPage;
+  if (idx < 0 || idx >= L || j >= p.bt_stride) {
+    atomicOr(p.status, (uint32_t)MLA_DEVICE_STATUS_BOUNDS);
+    return -1;
   }
-  int pg[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    const bool in = idx[e] >= 0 && idx[e] < L;
-    const int j = in ? idx[e] / kPage : 0;
-    const bool jin = in && j < p.bt_stride;
-    if (idx[e] != -1 && !jin) atomicOr(p.status, (uint32_t)MLA_DEVICE_STATUS_BOUNDS);
-    pg[e] = jin ? p.block_table[(size_t)b * p.bt_stride + j] : -1;
-    if (!jin) idx[e] = -1;
+  const int pg = p.block_table[(size_t)b * p.bt_stride + j];
+  if (pg < 0 || pg >= p.num_pages) {
+    atomicOr(p.status, (uint32_t)MLA_DEVICE_STATUS_BOUNDS);
+    return -1;
   }
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    const bool ok = idx[e] >= 0 && pg[e] >= 0 && pg[e] < p.num_pages;
-    if (idx[e] >= 0 && !ok) atomicOr(p.status, (uint32_t)MLA_DEVICE_STATUS_BOUNDS);
-    r[e] = ok ? pg[e] * kPage + idx[e] % kPage : oob;
-  }
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    uint32_t v = 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) v |= (r[4 * h + i] != oob ? 1u : 0u) << i;
-    v <<= 4 * (lane & 7);
-    v |= __shfl_xor_sync(0xffffffffu, v, 1);
-    v |= __shfl_xor_sync(0xffffffffu, v, 2);
-    v |= __shfl_xor_sync(0xffffffffu, v, 4);
-    if ((lane & 7) == 0) mask[4 * h + (lane >> 3)] = v;
-  }
-}
-
-// Sparse: the K slice j of this CTA's tile (lane l gathers rows 4l..4l+3).
-__device__ __forceinline__ void gather_k_slice(uint8_t* dst, const CUtensorMap* map, uint32_t bar, int j, int lane,
-                                               const int (&r)[8], uint32_t rank) {
-  const int a = rank ? r[4] : r[0], b = rank ? r[5] : r[1], c = rank ? r[6] : r[2], d = rank ? r[7] : r[3];
-  tma_gather4_pair(dst + 4 * lane * 128, map, bar, 64 * j, a, b, c, d);
-}
-
-// Sparse: the V slot (q, jd): keys 64q..64q+63 of the step, value dims
-// 256*jd + 128*rank + [0,128) as two 64-dim halves; lanes 16(q%2)..16(q%2)+15
-// hold the rows.
-template <int Q>
-__device__ __forceinline__ void gather_v_slot(uint8_t* dst, const CUtensorMap* map, uint32_t bar, int jd, int lane,
-                                              const int (&r)[8], uint32_t rank) {
-  const int l0 = 16 * (Q & 1);
-  if (lane >= l0 && lane < l0 + 16) {
-    const int e = 4 * (Q >> 1);
-    uint8_t* row = dst + (4 * (lane - l0)) * 128;
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh)
-      tma_gather4_pair(row + hh * 8192, map, bar, 256 * jd + 128 * (int)rank + 64 * hh, r[e], r[e + 1], r[e + 2],
-                       r[e + 3]);
-  }
+  return pg * kPage + idx % kPage;
 }
 
 template <bool SPARSE>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SPARSE ? kThreadsSparse : kThreads, 1)
     mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
                            const DecodeParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -236,7 +193,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&c->q_full, 1);
-    for (int i = 0; i < kN; ++i) mbar_init(&c->full[i], 1);
+    // paged: the even CTA's producer arrives with both CTAs' TMA bytes;
+    // sparse: this CTA's 128 loader threads (cp.async) + one forward from the odd CTA
+    for (int i = 0; i < kN; ++i) mbar_init(&c->full[i], SPARSE ? 129 : 1);
     for (int i = 0; i < 2; ++i) mbar_init(&c->p_full[i], 8);
     mbar_init(&c->o_free, 8);
     mbar_init(&c->drain, 1);
@@ -245,14 +204,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) mbar_init(&c->s_full[i], 1);
     for (int i = 0; i < 2; ++i) mbar_init(&c->o_done[i], 1);
     mbar_init(&c->v_fix, 1);
-    for (int i = 0; i < 4; ++i) mbar_init(&c->m_full[i], 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&c->m_full[i], 4);
+    for (int i = 0; i < kN; ++i) mbar_init(&c->v_loc[i], 128);
     mbar_init(&c->grp_sm, 128);
     c->abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tm_q);
-    tma_prefetch_desc(&tm_kv);
+    if (!SPARSE) tma_prefetch_desc(&tm_kv);  // the sparse path gathers rows with cp.async
   }
   if (warp == 1) {
     tmem_alloc_pair(&c->tmem_base, kTmemCols);
@@ -270,8 +230,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer: Q, then the ring in order
     int sc = 0, pi = 0, q_issued = 0, fixc = 0;
-    int gk = 0, gv = 0;        // steps whose K / V this warp has issued (all pieces)
-    int rs0[8], rs1[8];        // sparse: cache rows of steps with even / odd gk
     bool stop = false;
     while (!stop && it.next(pc)) {
       if (lane == 0) {
@@ -289,30 +247,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int req = unit_req(p, pc.unit);
       const int Ls = p.seqlens[req];
       const int npg = (Ls + kPage - 1) / kPage;
-      const int nsteps = (pc.t1 - pc.t0 + 1) >> 1;
+      const int nsteps = SPARSE ? 0 : (pc.t1 - pc.t0 + 1) >> 1;  // sparse rows: loader warps
       PageWindow pw;
-      for (int h = 0; h <= 2 * nsteps && !stop; ++h) {
+      for (int h = 0; nsteps > 0 && h <= 2 * nsteps && !stop; ++h) {
         if (!ring_entry_exists(h, nsteps)) continue;
         const int k = pc.t0 + 2 * ring_entry_step(h);
-        if (ring_entry_is_k(h) && SPARSE) {
-          if (gk & 1) resolve_sparse_step(p, pc.unit, req, Ls, k, pc.t1, lane, rs1, c->vmask[gk & 3]);
-          else resolve_sparse_step(p, pc.unit, req, Ls, k, pc.t1, lane, rs0, c->vmask[gk & 3]);
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&c->m_full[gk & 3]);  // the softmax of this step reads the mask
-          for (int j = 0; j < 9; ++j, ++sc) {
-            const int slot = sc % kN;
-            bool ok = true;
-            if (lane == 0) ok = pwait(pr, &c->empty[slot], ((sc / kN) & 1) ^ 1, p);
-            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-            if (!ok) { stop = true; break; }
-            const uint32_t bar = map_to_rank(smem_u32(&c->full[slot]), 0);
-            if (lane == 0 && pr.leader) mbar_arrive_expect_tx(&c->full[slot], 2 * kSlot);
-            __syncwarp();
-            if (gk & 1) gather_k_slice(sRing + slot * kSlot, &tm_kv, bar, j, lane, rs1, pr.rank);
-            else gather_k_slice(sRing + slot * kSlot, &tm_kv, bar, j, lane, rs0, pr.rank);
-          }
-          ++gk;
-        } else if (ring_entry_is_k(h)) {
+        if (ring_entry_is_k(h)) {
           // own tile; past the piece's end the pair's other tile is loaded
           // again (its keys are masked)
           const int t = (k + (int)pr.rank < pc.t1) ? k + (int)pr.rank : k;
@@ -322,7 +262,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           int pa = pw.get(p, req, 2 * t, npg, lane);
           int pb = pw.get(p, req, 2 * t + 1, npg, lane);
           if (pb < 0) pb = pa;
-          ++gk;
           for (int j = 0; j < 9; ++j, ++sc) {
             const int slot = sc % kN;
             uint8_t* dst = sRing + slot * kSlot;
@@ -339,37 +278,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
             if (!ok) { stop = true; break; }
           }
-        } else if (SPARSE) {
-          // V of the step: slot (q, jd) = keys 64q..64q+63, value dims
-          // 256*jd + 128*rank + [0,128) as two 64-dim halves
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-#pragma unroll
-            for (int jd = 0; jd < 2; ++jd) {
-              const int slot = sc % kN;
-              bool ok = !stop;
-              if (lane == 0 && ok) ok = pwait(pr, &c->empty[slot], ((sc / kN) & 1) ^ 1, p);
-              ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-              if (!ok) { stop = true; continue; }
-              const uint32_t bar = map_to_rank(smem_u32(&c->full[slot]), 0);
-              if (lane == 0 && pr.leader) mbar_arrive_expect_tx(&c->full[slot], 2 * kSlot);
-              __syncwarp();
-              uint8_t* dst = sRing + slot * kSlot;
-              if (gv & 1) {
-                if (q == 0) gather_v_slot<0>(dst, &tm_kv, bar, jd, lane, rs1, pr.rank);
-                if (q == 1) gather_v_slot<1>(dst, &tm_kv, bar, jd, lane, rs1, pr.rank);
-                if (q == 2) gather_v_slot<2>(dst, &tm_kv, bar, jd, lane, rs1, pr.rank);
-                if (q == 3) gather_v_slot<3>(dst, &tm_kv, bar, jd, lane, rs1, pr.rank);
-              } else {
-                if (q == 0) gather_v_slot<0>(dst, &tm_kv, bar, jd, lane, rs0, pr.rank);
-                if (q == 1) gather_v_slot<1>(dst, &tm_kv, bar, jd, lane, rs0, pr.rank);
-                if (q == 2) gather_v_slot<2>(dst, &tm_kv, bar, jd, lane, rs0, pr.rank);
-                if (q == 3) gather_v_slot<3>(dst, &tm_kv, bar, jd, lane, rs0, pr.rank);
-              }
-              ++sc;
-            }
-          }
-          ++gv;
         } else {
           // V: slot (q, jd) = page q of the step (tile k + q/2, page half
           // q%2), value dims 256*jd + 128*rank + [0,128) as two 64-dim halves
@@ -430,6 +338,107 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (q_issued > 0) mbar_wait_cluster(&c->q_full, (uint32_t)((q_issued - 1) & 1), p.timeout_ns);
       for (int i = sc > kN ? sc - kN : 0; i < sc; ++i)
         mbar_wait_cluster(&c->full[i % kN], (uint32_t)((i / kN) & 1), p.timeout_ns);
+    }
+    __syncwarp();
+  } else if (SPARSE && (warp == 2 || warp == 3 || warp >= 8)) {
+    // ------------------------------------------------------------ sparse: cp.async row gathers
+    // Thread lt (0..127) owns index slot lt of each 128-slot tile: it copies
+    // that key's row into the K slices of this CTA's tile and, for the V
+    // slots, the keys 64q..64q+63 of the step that include it. Ignored slots
+    // are zero-filled. Ring order as for the paged cache.
+    const int lw = warp < 4 ? warp - 2 : warp - 6;
+    const int lt = 32 * lw + lane;
+    const uint8_t* cache = static_cast<const uint8_t*>(p.kcache);
+    int sc = 0, gk = 0, gv = 0;
+    int ra0 = -1, rb0 = -1, ra1 = -1, rb1 = -1;  // rows of tiles k, k+1 of steps with even / odd gk
+    bool stop = false;
+    while (!stop && it.next(pc)) {
+      const int b = unit_req(p, pc.unit);
+      const int L = p.seqlens[b];
+      const int nsteps = (pc.t1 - pc.t0 + 1) >> 1;
+      for (int h = 0; h <= 2 * nsteps && !stop; ++h) {
+        if (!ring_entry_exists(h, nsteps)) continue;
+        const int k = pc.t0 + 2 * ring_entry_step(h);
+        if (ring_entry_is_k(h)) {
+          const int ra = sparse_slot_row(p, pc.unit, b, L, kTile * k + lt, pc.t1);
+          const int rb = sparse_slot_row(p, pc.unit, b, L, kTile * (k + 1) + lt, pc.t1);
+          if (gk & 1) { ra1 = ra; rb1 = rb; } else { ra0 = ra; rb0 = rb; }
+          const uint32_t va = __ballot_sync(0xffffffffu, ra >= 0), vb = __ballot_sync(0xffffffffu, rb >= 0);
+          if (lane == 0) {
+            c->vmask[gk & 3][lw] = va;
+            c->vmask[gk & 3][4 + lw] = vb;
+            mbar_arrive(&c->m_full[gk & 3]);  // the softmax of this step reads the mask
+          }
+          // K slice j of this CTA's tile: this warp copies its 32 keys' rows,
+          // 8 lanes per 128-B row (row pointers of key 4i + lane/8 by shuffle)
+          const int row = pr.rank ? rb : ra;
+          const int ch = lane & 7;
+          for (int j = 0; j < 9; ++j, ++sc) {
+            const int slot = sc % kN;
+            bool ok = true;
+            if (lane == 0) ok = pwait(pr, &c->empty[slot], ((sc / kN) & 1) ^ 1, p);
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok) { stop = true; break; }
+            uint8_t* base = sRing + slot * kSlot + (32 * lw) * 128;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const int key = 4 * i + (lane >> 3);  // key within this warp's 32
+              const int r = __shfl_sync(0xffffffffu, row, key);
+              const uint8_t* src = cache + (size_t)(r >= 0 ? r : 0) * (kDqk * 2) + 128 * j + 16 * ch;
+              cp_async16(base + key * 128 + ((ch ^ (key & 7)) << 4), src, r >= 0 ? 16u : 0u);
+            }
+            cp_async_commit();
+            cp_async_mbar_arrive_noinc(pr.leader ? &c->full[slot] : &c->v_loc[slot]);
+          }
+          ++gk;
+        } else {
+          const int ra = (gv & 1) ? ra1 : ra0, rb = (gv & 1) ? rb1 : rb0;
+          for (int q = 0; q < 4 && !stop; ++q) {
+            // V slot (q, jd): keys 64q..64q+63 of the step belong to warps
+            // 2(q%2) and 2(q%2)+1 (lw); 16 lanes per key row (two 128-B halves)
+            const bool mine = (lw >> 1) == (q & 1);
+            const int row = (q >> 1) ? rb : ra;
+            const int ch = lane & 7, hh = (lane >> 3) & 1;
+            for (int jd = 0; jd < 2; ++jd, ++sc) {
+              const int slot = sc % kN;
+              bool ok = true;
+              if (lane == 0) ok = pwait(pr, &c->empty[slot], ((sc / kN) & 1) ^ 1, p);
+              ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+              if (!ok) { stop = true; break; }
+              if (mine) {
+                uint8_t* base = sRing + slot * kSlot + hh * 8192 + (32 * (lw & 1)) * 128;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                  const int key = 2 * i + (lane >> 4);  // key within this warp's 32
+                  const int r = __shfl_sync(0xffffffffu, row, key);
+                  const uint8_t* src = cache + (size_t)(r >= 0 ? r : 0) * (kDqk * 2) + 256 * (int)pr.rank + 512 * jd +
+                                       128 * hh + 16 * ch;
+                  const int vrow = 32 * (lw & 1) + key;  // row within the 64-key slot
+                  cp_async16(base + key * 128 + ((ch ^ (vrow & 7)) << 4), src, r >= 0 ? 16u : 0u);
+                }
+                cp_async_commit();
+              }
+              cp_async_mbar_arrive_noinc(pr.leader ? &c->full[slot] : &c->v_loc[slot]);
+            }
+          }
+          ++gv;
+        }
+      }
+    }
+    cp_async_commit();
+    cp_async_wait<0>();  // no copy may land after the CTA has finished
+  } else if (SPARSE && warp == 1 && !pr.leader) {
+    // ------------------------------------------------------------ sparse, odd CTA: forward slot completions
+    if (lane == 0) {
+      int sc = 0;
+      bool stop = false;
+      while (!stop && it.next(pc)) {
+        const int nslots = 17 * ((pc.t1 - pc.t0 + 1) >> 1);  // 9 K slices + 8 V slots per step
+        for (int i = 0; i < nslots; ++i, ++sc) {
+          if (!pwait(pr, &c->v_loc[sc % kN], (sc / kN) & 1, p)) { stop = true; break; }
+          arrive_leader(pr, &c->full[sc % kN]);
+        }
+      }
     }
     __syncwarp();
   } else if (warp == 1 && pr.leader) {
@@ -680,7 +689,7 @@ cudaError_t launch_decode_pair(const CUtensorMap& tq, const CUtensorMap& tkv, co
   auto kern = sparse ? pair::mla_decode_pair_kernel<true> : pair::mla_decode_pair_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  kern<<<2 * parts, pair::kThreads, smem, stream>>>(tq, tkv, p);
+  kern<<<2 * parts, sparse ? pair::kThreadsSparse : pair::kThreads, smem, stream>>>(tq, tkv, p);
   return cudaGetLastError();
 }
 
