@@ -100,8 +100,8 @@ __device__ __forceinline__ bool group_sync(Ctrl* c, uint64_t* bar, uint32_t& pha
 // as one group and retires the slot it issued kLag slots earlier: wait for
 // that group, convert it (FP8), fence the generic-proxy writes for the tensor
 // core, arrive on the slot's full barrier (count 32).
-// Lane t copies tokens t + 32q of a 128-token tile (q = 0..3); a V slot holds
-// the 64 tokens of one page, so lane t copies its tokens t and t + 32 there.
+// Lane t resolves the source rows of tokens t + 32q of a 128-token tile
+// (q = 0..3); the copies themselves put several lanes on each row.
 constexpr int kGatherLanes = 32;
 
 struct GatherRing {
@@ -111,49 +111,53 @@ struct GatherRing {
   int nslots;
 };
 
+// Pointer held by lane `src` of the warp.
+__device__ __forceinline__ const uint8_t* shfl_ptr(const uint8_t* v, int src) {
+  return reinterpret_cast<const uint8_t*>(
+      __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(v), src));
+}
+
+// FP8: converts the staged codes of a retired slot in place. Four lanes share
+// a row (reads of a row complete before any lane overwrites it).
 template <int MODE, bool KGROUP>
 __device__ __forceinline__ void retire_slot(const GatherRing& g, int seq, int t) {
   const int slot = seq % g.nslots;
   uint8_t* s = g.base + slot * kSlot;
   if (MODE == kModeFp8) {
+    __syncwarp();  // every lane's copies of this slot are complete and visible
     if (KGROUP) {
       const int j = seq % 9;
-      if (j != 8) {  // latent slice: codes in bytes [0,64) and scales in [64,80) of the row
-#pragma unroll 1
-        for (int q = 0; q < 4; ++q) {
-          const int row = t + 32 * q;
-          const uint4* raw = reinterpret_cast<const uint4*>(s + row * 128);
-          uint4 cw[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) cw[i] = raw[i];
-          const float scale = pick4(*reinterpret_cast<const float4*>(s + row * 128 + 64), j >> 1);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            uint4 lo, hi;
-            dequant16(cw[i], scale, lo, hi);
-            *reinterpret_cast<uint4*>(sw128(s, row, 2 * i)) = lo;
-            *reinterpret_cast<uint4*>(sw128(s, row, 2 * i + 1)) = hi;
-          }
+      if (j != 8) {  // latent slice: codes in bytes [0,64) and scales in [64,80) of each row
+#pragma unroll 4
+        for (int i = 0; i < 16; ++i) {
+          const int r = 8 * i + (t >> 2), cc = t & 3;
+          const uint4 cw = *reinterpret_cast<const uint4*>(s + r * 128 + 16 * cc);
+          const float scale = reinterpret_cast<const float*>(s + r * 128 + 64)[j >> 1];
+          __syncwarp();
+          uint4 lo, hi;
+          dequant16(cw, scale, lo, hi);
+          *reinterpret_cast<uint4*>(sw128(s, r, 2 * cc)) = lo;
+          *reinterpret_cast<uint4*>(sw128(s, r, 2 * cc + 1)) = hi;
         }
       }
-    } else {  // V slot: codes in half-0 row, scales at the start of the half-1 row
+    } else {  // V slot: codes in the half-0 row, scales at the start of the half-1 row
       const int m = (seq >> 1) & 3;
-#pragma unroll 1
-      for (int q = 0; q < 2; ++q) {
-        const int row = t + 32 * q;
-        const uint4* raw = reinterpret_cast<const uint4*>(s + row * 128);
-        uint4 cw[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) cw[i] = raw[i];
-        const float scale = pick4(*reinterpret_cast<const float4*>(s + 8192 + row * 128), m);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          uint4 lo, hi;
-          dequant16(cw[i], scale, lo, hi);
-          uint8_t* half = s + (i >> 2) * 8192;
-          *reinterpret_cast<uint4*>(sw128(half, row, 2 * (i & 3))) = lo;
-          *reinterpret_cast<uint4*>(sw128(half, row, 2 * (i & 3) + 1)) = hi;
-        }
+#pragma unroll 4
+      for (int i = 0; i < 8; ++i) {
+        const int r = 8 * i + (t >> 2), c4 = t & 3;  // codes 32*c4 .. 32*c4+31 of row r
+        const uint4 cw0 = *reinterpret_cast<const uint4*>(s + r * 128 + 32 * c4);
+        const uint4 cw1 = *reinterpret_cast<const uint4*>(s + r * 128 + 32 * c4 + 16);
+        const float scale = reinterpret_cast<const float*>(s + 8192 + r * 128)[m];
+        __syncwarp();
+        uint8_t* half = s + (c4 >> 1) * 8192;
+        const int c0 = 4 * (c4 & 1);
+        uint4 lo, hi;
+        dequant16(cw0, scale, lo, hi);
+        *reinterpret_cast<uint4*>(sw128(half, r, c0)) = lo;
+        *reinterpret_cast<uint4*>(sw128(half, r, c0 + 1)) = hi;
+        dequant16(cw1, scale, lo, hi);
+        *reinterpret_cast<uint4*>(sw128(half, r, c0 + 2)) = lo;
+        *reinterpret_cast<uint4*>(sw128(half, r, c0 + 3)) = hi;
       }
     }
   }
@@ -172,7 +176,9 @@ __device__ void gather_group(const DecodeParams& p, Ctrl* c, PieceIter& it, cons
     const int req = unit_req(p, unit);
     const int npg = (MODE == kModeSparse) ? 0 : (p.seqlens[req] + kPage - 1) / kPage;
     for (int k = pc.t0; k < pc.t1 && !stop; ++k) {
-      // source rows of tokens t + 32q of the tile (q = 0..3)
+      // source rows of tokens t + 32q of the tile (q = 0..3); the copies
+      // below are coalesced (several lanes per row), so row pointers move
+      // between lanes by shuffle
       const uint8_t* src[4];
       uint32_t ok[4];
 #pragma unroll
@@ -194,36 +200,46 @@ __device__ void gather_group(const DecodeParams& p, Ctrl* c, PieceIter& it, cons
         const int slot = seq % g.nslots;
         uint8_t* s = g.base + slot * kSlot;
         if (!timed_wait(c, &g.empty[slot], ((seq / g.nslots) & 1) ^ 1, p)) { stop = true; break; }
-        if (KGROUP) {  // slice j (64 dims) of the four tokens
+        if (KGROUP) {
+          if (MODE == kModeSparse || j == 8) {  // bf16 128-B row slice: 8 lanes per row
+            const int off = MODE == kModeSparse ? 128 * j : 528;
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int row = t + 32 * q;
-            if (MODE == kModeSparse) {
-#pragma unroll
-              for (int ch = 0; ch < 8; ++ch) cp_async16(sw128(s, row, ch), src[q] + 128 * j + 16 * ch, ok[q]);
-            } else if (j == 8) {  // RoPE dims: bf16 straight into place
-#pragma unroll
-              for (int ch = 0; ch < 8; ++ch) cp_async16(sw128(s, row, ch), src[q] + 528 + 16 * ch, 16u);
-            } else {  // latent codes + scales into the row, converted at retire
-#pragma unroll
-              for (int ch = 0; ch < 4; ++ch) cp_async16(s + row * 128 + 16 * ch, src[q] + 64 * j + 16 * ch, 16u);
-              cp_async16(s + row * 128 + 64, src[q] + 512, 16u);
+            for (int i = 0; i < 32; ++i) {
+              const int r = 4 * i + (t >> 3), ch = t & 7;
+              const uint8_t* sp = shfl_ptr(src[i >> 3], r & 31);
+              const uint32_t nb = __shfl_sync(0xffffffffu, ok[i >> 3], r & 31);
+              cp_async16(sw128(s, r, ch), sp + off + 16 * ch, nb);
             }
+          } else {  // FP8 latent slice j: codes (64 B, 4 lanes per row) and scales, converted at retire
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int r = 8 * i + (t >> 2), cc = t & 3;
+              cp_async16(s + r * 128 + 16 * cc, shfl_ptr(src[i >> 2], r & 31) + 64 * j + 16 * cc, 16u);
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) cp_async16(s + (t + 32 * q) * 128 + 64, src[q] + 512, 16u);
           }
-        } else {  // V slot j: value dims 128*(j/2).., page half h = j%2, tokens t and t+32 of it
+        } else {  // V slot j: value dims 128*(j/2).., page half h = j%2 (tokens 64h..64h+63)
           const int m = j >> 1, h = j & 1;
+          const uint8_t* s0 = h ? src[2] : src[0];
+          const uint8_t* s1 = h ? src[3] : src[1];
+          const uint32_t ok0 = h ? ok[2] : ok[0], ok1 = h ? ok[3] : ok[1];
+          if (MODE == kModeSparse) {  // 256 B per row in two 128-B halves: 16 lanes per row
 #pragma unroll
-          for (int qq = 0; qq < 2; ++qq) {
-            const int q = 2 * h + qq, row = t + 32 * qq;
-            if (MODE == kModeSparse) {
-#pragma unroll
-              for (int ch = 0; ch < 16; ++ch)
-                cp_async16(sw128(s + (ch >> 3) * 8192, row, ch & 7), src[q] + 256 * m + 16 * ch, ok[q]);
-            } else {
-#pragma unroll
-              for (int ch = 0; ch < 8; ++ch) cp_async16(s + row * 128 + 16 * ch, src[q] + 128 * m + 16 * ch, 16u);
-              cp_async16(s + 8192 + row * 128, src[q] + 512, 16u);
+            for (int i = 0; i < 32; ++i) {
+              const int rr = 2 * i + (t >> 4), hh = (t >> 3) & 1, ch = t & 7;
+              const uint8_t* sp = shfl_ptr((i >> 4) ? s1 : s0, rr & 31);
+              const uint32_t nb = __shfl_sync(0xffffffffu, (i >> 4) ? ok1 : ok0, rr & 31);
+              cp_async16(sw128(s + hh * 8192, rr, ch), sp + 256 * m + 128 * hh + 16 * ch, nb);
             }
+          } else {  // FP8: codes (128 B, 8 lanes per row) in the half-0 row, scales at the half-1 row start
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int rr = 4 * i + (t >> 3), ch = t & 7;
+              cp_async16(s + rr * 128 + 16 * ch, shfl_ptr((i >> 3) ? s1 : s0, rr & 31) + 128 * m + 16 * ch, 16u);
+            }
+            cp_async16(s + 8192 + t * 128, s0 + 512, 16u);
+            cp_async16(s + 8192 + (t + 32) * 128, s1 + 512, 16u);
           }
         }
         cp_async_commit();
