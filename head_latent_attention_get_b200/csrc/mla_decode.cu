@@ -23,11 +23,11 @@
 // the PV product rather than held across the softmax, which keeps the rings
 // deep enough to cover the load latency.
 //
-// Warp roles (256 threads; 320 with the FP8 cache or sparse indices):
+// Warp roles (256 threads; 512 with the FP8 cache or sparse indices):
 //   0 Q (and, bf16 paged, K slices) via TMA   1 S issuer (+ TMEM alloc)
 //   2 O issuer                                 3 V slots via TMA (bf16 paged)
 //   4-7 softmax + epilogue (row r = 16*(warp-4) + lane, lanes 0-15)
-//   8 K gather warp, 9 V gather warp (FP8 / sparse): cp.async copies
+//   8-11 K gather warps, 12-15 V gather warps (FP8 / sparse): cp.async copies
 //       software-pipelined three slots deep; FP8 codes are converted in place.
 // Every mbarrier wait is bounded; on timeout the CTA records
 // MLA_DEVICE_STATUS_TIMEOUT, stops issuing work, waits (bounded) for its own
@@ -95,14 +95,17 @@ __device__ __forceinline__ bool group_sync(Ctrl* c, uint64_t* bar, uint32_t& pha
 }
 
 // ============================================================================ gather groups
-// FP8 and sparse modes: one warp fills the K ring and one warp the V ring with
-// 16-byte cp.async copies. Each lane issues the copies of a slot, commits them
-// as one group and retires the slot it issued kLag slots earlier: wait for
-// that group, convert it (FP8), fence the generic-proxy writes for the tensor
-// core, arrive on the slot's full barrier (count 32).
-// Lane t resolves the source rows of tokens t + 32q of a 128-token tile
-// (q = 0..3); the copies themselves put several lanes on each row.
-constexpr int kGatherLanes = 32;
+// FP8 and sparse modes: four warps fill the K ring and four the V ring with
+// 16-byte cp.async copies. Warp lw of a group owns a quarter of every slot's
+// rows (K: tile rows 32lw..32lw+31; V: page rows 16lw..16lw+15), lane t the
+// source row of one of them; the copies put 4-16 lanes on each row (row
+// pointers by shuffle), FP8 codes are converted in place with four lanes per
+// row. Each warp issues a slot's copies, commits them as one group and retires
+// the slot it issued kLag slots earlier: wait for that group, convert it
+// (FP8), fence the generic-proxy writes for the tensor core, arrive on the
+// slot's full barrier (count 32 x 4 warps).
+constexpr int kGatherWarps = 4;
+constexpr int kGatherThreads = 32 * kGatherWarps;
 
 struct GatherRing {
   uint64_t* full;
@@ -117,10 +120,10 @@ __device__ __forceinline__ const uint8_t* shfl_ptr(const uint8_t* v, int src) {
       __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(v), src));
 }
 
-// FP8: converts the staged codes of a retired slot in place. Four lanes share
-// a row (reads of a row complete before any lane overwrites it).
+// FP8: converts this warp's rows of a retired slot in place, four lanes per
+// row (every lane reads a row before any lane overwrites it).
 template <int MODE, bool KGROUP>
-__device__ __forceinline__ void retire_slot(const GatherRing& g, int seq, int t) {
+__device__ __forceinline__ void retire_slot(const GatherRing& g, int seq, int lw, int t) {
   const int slot = seq % g.nslots;
   uint8_t* s = g.base + slot * kSlot;
   if (MODE == kModeFp8) {
@@ -128,9 +131,9 @@ __device__ __forceinline__ void retire_slot(const GatherRing& g, int seq, int t)
     if (KGROUP) {
       const int j = seq % 9;
       if (j != 8) {  // latent slice: codes in bytes [0,64) and scales in [64,80) of each row
-#pragma unroll 4
-        for (int i = 0; i < 16; ++i) {
-          const int r = 8 * i + (t >> 2), cc = t & 3;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = 32 * lw + 8 * i + (t >> 2), cc = t & 3;
           const uint4 cw = *reinterpret_cast<const uint4*>(s + r * 128 + 16 * cc);
           const float scale = reinterpret_cast<const float*>(s + r * 128 + 64)[j >> 1];
           __syncwarp();
@@ -142,9 +145,9 @@ __device__ __forceinline__ void retire_slot(const GatherRing& g, int seq, int t)
       }
     } else {  // V slot: codes in the half-0 row, scales at the start of the half-1 row
       const int m = (seq >> 1) & 3;
-#pragma unroll 4
-      for (int i = 0; i < 8; ++i) {
-        const int r = 8 * i + (t >> 2), c4 = t & 3;  // codes 32*c4 .. 32*c4+31 of row r
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int r = 16 * lw + 8 * i + (t >> 2), c4 = t & 3;  // codes 32*c4 .. 32*c4+31 of row r
         const uint4 cw0 = *reinterpret_cast<const uint4*>(s + r * 128 + 32 * c4);
         const uint4 cw1 = *reinterpret_cast<const uint4*>(s + r * 128 + 32 * c4 + 16);
         const float scale = reinterpret_cast<const float*>(s + 8192 + r * 128)[m];
@@ -165,8 +168,24 @@ __device__ __forceinline__ void retire_slot(const GatherRing& g, int seq, int t)
   mbar_arrive(&g.full[slot]);
 }
 
+// Source row of tile-relative token tt of tile k (FP8 record, or bf16 cache
+// row for sparse; ok = 0 for an ignored sparse slot, which is zero-filled).
 template <int MODE, bool KGROUP>
-__device__ void gather_group(const DecodeParams& p, Ctrl* c, PieceIter& it, const GatherRing& g, int t) {
+__device__ __forceinline__ const uint8_t* gather_src(const DecodeParams& p, int unit, int req, int npg, int k, int tt,
+                                                     uint32_t& ok) {
+  if (MODE == kModeSparse) {
+    const int row = sparse_row(p, unit, k * kTile + tt, KGROUP);
+    ok = row >= 0 ? 16u : 0u;
+    return static_cast<const uint8_t*>(p.kcache) + (size_t)(row >= 0 ? row : 0) * (kDqk * 2);
+  }
+  int pg = page_of(p, req, 2 * k + (tt >> 6), npg);
+  if (pg < 0) pg = page_of(p, req, 2 * k, npg);  // half tile: page A again (keys masked, values zero-filled later)
+  ok = 16u;
+  return p.kcache_fp8 + ((size_t)pg * kPage + (tt & 63)) * kFp8RecordBytes;
+}
+
+template <int MODE, bool KGROUP>
+__device__ void gather_group(const DecodeParams& p, Ctrl* c, PieceIter& it, const GatherRing& g, int lw, int t) {
   int seq = 0;       // slots issued
   int retired = 0;   // slots retired
   bool stop = false;
@@ -176,24 +195,17 @@ __device__ void gather_group(const DecodeParams& p, Ctrl* c, PieceIter& it, cons
     const int req = unit_req(p, unit);
     const int npg = (MODE == kModeSparse) ? 0 : (p.seqlens[req] + kPage - 1) / kPage;
     for (int k = pc.t0; k < pc.t1 && !stop; ++k) {
-      // source rows of tokens t + 32q of the tile (q = 0..3); the copies
-      // below are coalesced (several lanes per row), so row pointers move
-      // between lanes by shuffle
-      const uint8_t* src[4];
-      uint32_t ok[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int tt = t + 32 * q;
-        if (MODE == kModeSparse) {
-          const int row = sparse_row(p, unit, k * kTile + tt, KGROUP);
-          ok[q] = row >= 0 ? 16u : 0u;  // ignored slots are zero-filled
-          src[q] = static_cast<const uint8_t*>(p.kcache) + (size_t)(row >= 0 ? row : 0) * (kDqk * 2);
-        } else {
-          int pg = page_of(p, req, 2 * k + (tt >> 6), npg);
-          if (pg < 0) pg = page_of(p, req, 2 * k, npg);
-          ok[q] = 16u;
-          src[q] = p.kcache_fp8 + ((size_t)pg * kPage + (tt & 63)) * kFp8RecordBytes;
-        }
+      // K: lane t owns tile row 32lw + t; V: lane t (< 16) owns row 16lw + t
+      // of page h, i.e. tile row 64h + 16lw + t
+      uint32_t ok = 0, ok0 = 0, ok1 = 0;
+      const uint8_t* srcK = nullptr;
+      const uint8_t* srcV0 = nullptr;
+      const uint8_t* srcV1 = nullptr;
+      if (KGROUP) {
+        srcK = gather_src<MODE, KGROUP>(p, unit, req, npg, k, 32 * lw + t, ok);
+      } else {
+        srcV0 = gather_src<MODE, KGROUP>(p, unit, req, npg, k, 16 * lw + (t & 15), ok0);
+        srcV1 = gather_src<MODE, KGROUP>(p, unit, req, npg, k, 64 + 16 * lw + (t & 15), ok1);
       }
       const int slots_per_tile = KGROUP ? 9 : 8;
       for (int j = 0; j < slots_per_tile; ++j, ++seq) {
@@ -204,48 +216,43 @@ __device__ void gather_group(const DecodeParams& p, Ctrl* c, PieceIter& it, cons
           if (MODE == kModeSparse || j == 8) {  // bf16 128-B row slice: 8 lanes per row
             const int off = MODE == kModeSparse ? 128 * j : 528;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
+            for (int i = 0; i < 8; ++i) {
               const int r = 4 * i + (t >> 3), ch = t & 7;
-              const uint8_t* sp = shfl_ptr(src[i >> 3], r & 31);
-              const uint32_t nb = __shfl_sync(0xffffffffu, ok[i >> 3], r & 31);
-              cp_async16(sw128(s, r, ch), sp + off + 16 * ch, nb);
+              const uint32_t nb = __shfl_sync(0xffffffffu, ok, r);
+              cp_async16(sw128(s, 32 * lw + r, ch), shfl_ptr(srcK, r) + off + 16 * ch, nb);
             }
           } else {  // FP8 latent slice j: codes (64 B, 4 lanes per row) and scales, converted at retire
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
+            for (int i = 0; i < 4; ++i) {
               const int r = 8 * i + (t >> 2), cc = t & 3;
-              cp_async16(s + r * 128 + 16 * cc, shfl_ptr(src[i >> 2], r & 31) + 64 * j + 16 * cc, 16u);
+              cp_async16(s + (32 * lw + r) * 128 + 16 * cc, shfl_ptr(srcK, r) + 64 * j + 16 * cc, 16u);
             }
-#pragma unroll
-            for (int q = 0; q < 4; ++q) cp_async16(s + (t + 32 * q) * 128 + 64, src[q] + 512, 16u);
+            cp_async16(s + (32 * lw + t) * 128 + 64, srcK + 512, 16u);
           }
-        } else {  // V slot j: value dims 128*(j/2).., page half h = j%2 (tokens 64h..64h+63)
-          const int m = j >> 1, h = j & 1;
-          const uint8_t* s0 = h ? src[2] : src[0];
-          const uint8_t* s1 = h ? src[3] : src[1];
-          const uint32_t ok0 = h ? ok[2] : ok[0], ok1 = h ? ok[3] : ok[1];
+        } else {  // V slot j: value dims 128*(j/2).., page half h = j%2
+          const int m = j >> 1;
+          const uint8_t* sv = (j & 1) ? srcV1 : srcV0;
+          const uint32_t okv = (j & 1) ? ok1 : ok0;
           if (MODE == kModeSparse) {  // 256 B per row in two 128-B halves: 16 lanes per row
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int rr = 2 * i + (t >> 4), hh = (t >> 3) & 1, ch = t & 7;
-              const uint8_t* sp = shfl_ptr((i >> 4) ? s1 : s0, rr & 31);
-              const uint32_t nb = __shfl_sync(0xffffffffu, (i >> 4) ? ok1 : ok0, rr & 31);
-              cp_async16(sw128(s + hh * 8192, rr, ch), sp + 256 * m + 128 * hh + 16 * ch, nb);
+            for (int i = 0; i < 8; ++i) {
+              const int r = 2 * i + (t >> 4), hh = (t >> 3) & 1, ch = t & 7;
+              const uint32_t nb = __shfl_sync(0xffffffffu, okv, r);
+              cp_async16(sw128(s + hh * 8192, 16 * lw + r, ch), shfl_ptr(sv, r) + 256 * m + 128 * hh + 16 * ch, nb);
             }
           } else {  // FP8: codes (128 B, 8 lanes per row) in the half-0 row, scales at the half-1 row start
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int rr = 4 * i + (t >> 3), ch = t & 7;
-              cp_async16(s + rr * 128 + 16 * ch, shfl_ptr((i >> 3) ? s1 : s0, rr & 31) + 128 * m + 16 * ch, 16u);
+            for (int i = 0; i < 4; ++i) {
+              const int r = 4 * i + (t >> 3), ch = t & 7;
+              cp_async16(s + (16 * lw + r) * 128 + 16 * ch, shfl_ptr(sv, r) + 128 * m + 16 * ch, 16u);
             }
-            cp_async16(s + 8192 + t * 128, s0 + 512, 16u);
-            cp_async16(s + 8192 + (t + 32) * 128, s1 + 512, 16u);
+            if (t < 16) cp_async16(s + 8192 + (16 * lw + t) * 128, sv + 512, 16u);
           }
         }
         cp_async_commit();
         if (seq + 1 - retired > kLag) {
           cp_async_wait<kLag>();
-          retire_slot<MODE, KGROUP>(g, retired, t);
+          retire_slot<MODE, KGROUP>(g, retired, lw, t);
           ++retired;
         }
       }
@@ -254,7 +261,7 @@ __device__ void gather_group(const DecodeParams& p, Ctrl* c, PieceIter& it, cons
   cp_async_wait<0>();  // no copy may land after the CTA has finished
   if (!stop) {
     while (retired < seq) {
-      retire_slot<MODE, KGROUP>(g, retired, t);
+      retire_slot<MODE, KGROUP>(g, retired, lw, t);
       ++retired;
     }
   }
@@ -262,7 +269,7 @@ __device__ void gather_group(const DecodeParams& p, Ctrl* c, PieceIter& it, cons
 
 // ============================================================================ kernel
 template <int NR, int MODE>
-__global__ void __launch_bounds__(MODE == kModeBf16 ? 256 : 320, 1)
+__global__ void __launch_bounds__(MODE == kModeBf16 ? 256 : 256 + 2 * kGatherThreads, 1)
     mla_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
                       const DecodeParams p) {
   using L = Smem<NR>;
@@ -278,7 +285,7 @@ __global__ void __launch_bounds__(MODE == kModeBf16 ? 256 : 320, 1)
   const int part = blockIdx.x, rg = blockIdx.y;
   const int row0 = rg * kRowsPerCta;                    // first row of this CTA within a unit
   const int rows_here = min(kRowsPerCta, p.rows - row0);
-  constexpr uint32_t kFullCount = MODE == kModeBf16 ? 1 : kGatherLanes;
+  constexpr uint32_t kFullCount = MODE == kModeBf16 ? 1 : kGatherThreads;
 
   if (threadIdx.x == 0) {
     mbar_init(&c->q_full, 1);
@@ -383,12 +390,12 @@ __global__ void __launch_bounds__(MODE == kModeBf16 ? 256 : 320, 1)
     __syncwarp();
   } else if (MODE != kModeBf16 && warp >= 8) {
     // ------------------------------------------------------------ gather groups
-    if (warp == 8) {
+    if (warp < 8 + kGatherWarps) {
       const GatherRing g{c->k_full, c->k_empty, sK, kNK};
-      gather_group<MODE, true>(p, c, it, g, lane);
+      gather_group<MODE, true>(p, c, it, g, warp - 8, lane);
     } else {
       const GatherRing g{c->v_full, c->v_empty, sV, kNV};
-      gather_group<MODE, false>(p, c, it, g, lane);
+      gather_group<MODE, false>(p, c, it, g, warp - 8 - kGatherWarps, lane);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ S issuer
@@ -681,7 +688,7 @@ static cudaError_t launch_one(const CUtensorMap& tq, const CUtensorMap& tkv, con
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(parts, row_groups);
-  kern<<<grid, MODE == kModeBf16 ? 256 : 320, smem, stream>>>(tq, tkv, p);
+  kern<<<grid, MODE == kModeBf16 ? 256 : 256 + 2 * kGatherThreads, smem, stream>>>(tq, tkv, p);
   return cudaGetLastError();
 }
 
