@@ -3,7 +3,10 @@
 // one request's KV). Each split s of a unit holds its own softmax-normalised
 // partial output o_s and log-sum-exp lse_s over a disjoint subset of the keys:
 //   lse = ln sum_s exp(lse_s),   out = sum_s exp(lse_s - lse) * o_s.
-// One 128-thread block per (row, unit); each thread owns 4 of the 512 dims.
+// One block per (unit, chunk of 4 rows); a unit that was not split (its
+// piece wrote the output directly) costs the block one read. Each half-block
+// of 128 threads merges one row at a time, each thread owning 4 of the 512
+// dims.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -11,49 +14,56 @@
 
 namespace mla {
 
-constexpr int kCombineThreads = 128;
+constexpr int kCombineThreads = 256;
+constexpr int kCombineRows = 4;  // rows per block
 
 __global__ void __launch_bounds__(kCombineThreads) mla_combine_kernel(
     const float* __restrict__ part_lse, const float* __restrict__ part_o, const int32_t* __restrict__ split_ptr,
     int rows, __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
-  const int r = blockIdx.x, u = blockIdx.y;
-  const int s0 = split_ptr[u], n = split_ptr[u + 1] - s0;
-  if (n == 1) return;  // written directly by the decode kernel
-  const size_t orow = (size_t)u * rows + r;
-  const int d = threadIdx.x * 4;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  float L = -INFINITY;
-  if (n >= 2) {
-    float m = -INFINITY;
-    for (int s = 0; s < n; ++s) m = fmaxf(m, part_lse[(size_t)(s0 + s) * rows + r]);
-    if (m != -INFINITY) {
-      float sum = 0.f;
-      for (int s = 0; s < n; ++s) sum += expf(part_lse[(size_t)(s0 + s) * rows + r] - m);
-      L = m + logf(sum);
-      for (int s = 0; s < n; ++s) {
-        const float w = expf(part_lse[(size_t)(s0 + s) * rows + r] - L);
-        const float4 o = *reinterpret_cast<const float4*>(part_o + ((size_t)(s0 + s) * rows + r) * kDv + d);
-        acc.x += w * o.x; acc.y += w * o.y; acc.z += w * o.z; acc.w += w * o.w;
+  const int half = threadIdx.x >> 7;
+  const int d = (threadIdx.x & 127) * 4;
+  const int u = blockIdx.x;
+  {
+    const int s0 = split_ptr[u], n = split_ptr[u + 1] - s0;
+    if (n == 1) return;  // written directly by the decode kernel
+    const int r1 = min(rows, (int)(blockIdx.y + 1) * kCombineRows);
+    for (int r = blockIdx.y * kCombineRows + half; r < r1; r += 2) {
+      const size_t orow = (size_t)u * rows + r;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      float L = -INFINITY;  // no split at all: an empty key set (out 0, lse -inf)
+      if (n >= 2) {
+        float m = -INFINITY;
+        for (int s = 0; s < n; ++s) m = fmaxf(m, part_lse[(size_t)(s0 + s) * rows + r]);
+        if (m != -INFINITY) {
+          float sum = 0.f;
+          for (int s = 0; s < n; ++s) sum += expf(part_lse[(size_t)(s0 + s) * rows + r] - m);
+          L = m + logf(sum);
+          for (int s = 0; s < n; ++s) {
+            const float w = expf(part_lse[(size_t)(s0 + s) * rows + r] - L);
+            const float4 o = *reinterpret_cast<const float4*>(part_o + ((size_t)(s0 + s) * rows + r) * kDv + d);
+            acc.x += w * o.x; acc.y += w * o.y; acc.z += w * o.z; acc.w += w * o.w;
+          }
+        }
       }
+      __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+      __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+      uint2 packed;
+      packed.x = *reinterpret_cast<uint32_t*>(&lo);
+      packed.y = *reinterpret_cast<uint32_t*>(&hi);
+      *reinterpret_cast<uint2*>(out + orow * kDv + d) = packed;
+      if ((threadIdx.x & 127) == 0) lse[orow] = L;
     }
   }
-  __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
-  __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
-  uint2 packed;
-  packed.x = *reinterpret_cast<uint32_t*>(&lo);
-  packed.y = *reinterpret_cast<uint32_t*>(&hi);
-  *reinterpret_cast<uint2*>(out + orow * kDv + d) = packed;
-  if (threadIdx.x == 0) lse[orow] = L;
 }
 
 mla_status_t launch_combine(const void* workspace, int units, int rows, int parts, const int32_t* split_ptr,
                             void* out, float* lse, cudaStream_t stream) {
   const WsLayout w = ws_layout(units, rows, parts);
   const char* ws = static_cast<const char*>(workspace);
-  dim3 grid(rows, units);
+  const dim3 grid(units, (rows + kCombineRows - 1) / kCombineRows);
   mla_combine_kernel<<<grid, kCombineThreads, 0, stream>>>(
-      reinterpret_cast<const float*>(ws + w.lse_off), reinterpret_cast<const float*>(ws + w.o_off), split_ptr,
-      rows, static_cast<__nv_bfloat16*>(out), lse);
+      reinterpret_cast<const float*>(ws + w.lse_off), reinterpret_cast<const float*>(ws + w.o_off), split_ptr, rows,
+      static_cast<__nv_bfloat16*>(out), lse);
   return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
