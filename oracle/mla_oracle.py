@@ -16,6 +16,13 @@ b, query token i in [0, s_q) and head h:
   out      = sum_t exp(s_t - m) * row(t)[:512] / l        (V = first 512 dims)
   lse      = m + ln(l)                                    (natural log)
   empty T  : out = 0, lse = -inf   (the pages say nothing; chosen reading)
+  sink     : optional per-head logit sigma_h in the units of s_t; it joins the
+             softmax denominator as one more key whose value vector is zero:
+             m = max(max_t s_t, sigma), l = sum_t exp(s_t - m) + exp(sigma - m),
+             out as above over this l, lse = m + ln(l); with an empty T,
+             out = 0 and lse = sigma. (FlashInfer page, section 2: "an
+             optional per-head attention sink", sinks [num_heads] float32;
+             its exact use is not given, this is the plainest reading.)
 
 Passages followed:
   * FlashMLA-ETAP (gist.science summary), "핵심 메커니즘" (core mechanism):
@@ -123,21 +130,27 @@ def dequant_fp8_records(records) -> np.ndarray:
 # --------------------------------------------------------------------------
 # the attention definition
 # --------------------------------------------------------------------------
-def attend(q_rows, keys, scale, d_v=D_V):
+def attend(q_rows, keys, scale, d_v=D_V, sink=None):
     """softmax(scale * q_rows @ keys^T) @ keys[:, :d_v] and its natural-log LSE.
 
-    q_rows [R, d_qk], keys [T, d_qk] (T may be 0). Returns (out [R, d_v],
-    lse [R]). Empty key set: out 0, lse -inf.
+    q_rows [R, d_qk], keys [T, d_qk] (T may be 0), sink None or [R] logits
+    (an extra zero-value key per row). Returns (out [R, d_v], lse [R]).
+    Empty key set: out 0, lse -inf (lse = sink with a sink).
     """
     q_rows = np.asarray(q_rows, dtype=np.float64)
     keys = np.asarray(keys, dtype=np.float64)
     R = q_rows.shape[0]
+    sk = None if sink is None else np.asarray(sink, dtype=np.float64).reshape(R)
     if keys.shape[0] == 0:
-        return np.zeros((R, d_v)), np.full(R, -np.inf)
+        return np.zeros((R, d_v)), (np.full(R, -np.inf) if sk is None else sk.copy())
     s = scale * (q_rows @ keys.T)                        # [R, T]
     m = s.max(axis=1, keepdims=True)
+    if sk is not None:
+        m = np.maximum(m, sk[:, None])
     e = np.exp(s - m)
     l = e.sum(axis=1, keepdims=True)
+    if sk is not None:
+        l = l + np.exp(sk[:, None] - m)
     out = (e @ keys[:, :d_v]) / l
     lse = m[:, 0] + np.log(l[:, 0])
     return out, lse
@@ -167,7 +180,7 @@ def cache_to_f64(kcache) -> np.ndarray:
 
 
 def decode_dense(q, cache_f64, block_table, cache_seqlens, scale, causal,
-                 d_v=D_V, requests=None):
+                 d_v=D_V, requests=None, sink=None):
     """Dense paged MLA decode. q [B, s_q, h_q, d_qk] (fp64 values).
 
     Returns out [B, s_q, h_q, d_v] and lse [B, s_q, h_q] (requests not in
@@ -186,7 +199,7 @@ def decode_dense(q, cache_f64, block_table, cache_seqlens, scale, causal,
             n = L
             if causal:
                 n = max(0, min(L, L - s_q + i + 1))
-            o, l_ = attend(q[b, i], keys_all[:n], scale, d_v)
+            o, l_ = attend(q[b, i], keys_all[:n], scale, d_v, sink)
             out[b, i], lse[b, i] = o, l_
     return out, lse
 
@@ -204,7 +217,7 @@ def sparse_key_positions(index_row, seqlen):
 
 
 def decode_sparse(q, cache_f64, block_table, cache_seqlens, indices, scale,
-                  d_v=D_V, requests=None):
+                  d_v=D_V, requests=None, sink=None):
     """Token-sparse paged MLA decode; key set per (b, i) from indices[b, i]."""
     q = np.asarray(q, dtype=np.float64)
     B, s_q, h_q, _ = q.shape
@@ -217,22 +230,27 @@ def decode_sparse(q, cache_f64, block_table, cache_seqlens, indices, scale,
         for i in range(s_q):
             pos, _, _ = sparse_key_positions(idx[b, i], int(lens[b]))
             keys = gather_rows(cache_f64, bt[b], pos)
-            o, l_ = attend(q[b, i], keys, scale, d_v)
+            o, l_ = attend(q[b, i], keys, scale, d_v, sink)
             out[b, i], lse[b, i] = o, l_
     return out, lse
 
 
-def combine(o_parts, lse_parts):
+def combine(o_parts, lse_parts, sink=None):
     """Merge attention results of disjoint key subsets (split-KV reduction).
 
     o_parts [n, R, d] (each normalised over its own subset), lse_parts [n, R].
     L = ln sum_s exp(lse_s); out = sum_s exp(lse_s - L) o_s. All parts empty:
-    out 0, lse -inf.
+    out 0, lse -inf. A sink [R] enters as one more part with lse = sink and
+    a zero output.
     (FlashInfer PR #5443 analysis, section 3: a split-KV combine kernel merges
     the partial results of CTAs that split one request's KV.)
     """
     o_parts = np.asarray(o_parts, dtype=np.float64)
     lse_parts = np.asarray(lse_parts, dtype=np.float64)
+    if sink is not None:
+        sk = np.asarray(sink, dtype=np.float64).reshape(1, -1)
+        o_parts = np.concatenate([o_parts, np.zeros((1,) + o_parts.shape[1:])], axis=0)
+        lse_parts = np.concatenate([lse_parts, sk], axis=0)
     mx = lse_parts.max(axis=0)
     finite = np.isfinite(mx)
     mxs = np.where(finite, mx, 0.0)
@@ -253,8 +271,9 @@ def reference_decode(inp, requests=None):
     """Run the oracle on a workloads.DecodeInputs; returns (out, lse) fp64."""
     w = inp.workload
     q, cache = inputs_to_f64(inp)
+    sink = None if getattr(inp, "sink", None) is None else inp.sink.double().numpy()
     if w.topk:
         return decode_sparse(q, cache, inp.block_table.numpy(), inp.cache_seqlens.numpy(),
-                             inp.indices.numpy(), w.scale, requests=requests)
+                             inp.indices.numpy(), w.scale, requests=requests, sink=sink)
     return decode_dense(q, cache, inp.block_table.numpy(), inp.cache_seqlens.numpy(),
-                        w.scale, w.causal, requests=requests)
+                        w.scale, w.causal, requests=requests, sink=sink)

@@ -324,3 +324,117 @@ def check_golden_two_tokens(decode_dense):
     nz = set(int(k) for k in g["out_sparse"])
     assert all(out[0, 0, 0, j] == 0 for j in range(512) if j not in nz)
     _close(lse[0, 0, 0], g["lse"], 1e-15)
+
+
+# ---------------------------------------------------------------- attention sink
+def _mp_attend_sink(q_rows, keys, scale, d_v, sink):
+    """50-digit brute force with one extra logit per row that carries no value."""
+    outs, lses = [], []
+    for r in range(len(q_rows)):
+        s = [mpmath.mpf(scale) * mpmath.fsum(mpmath.mpf(float(a)) * mpmath.mpf(float(b))
+                                             for a, b in zip(q_rows[r], k)) for k in keys]
+        sg = mpmath.mpf(float(sink[r]))
+        m = max(s + [sg])
+        e = [mpmath.exp(x - m) for x in s]
+        l = mpmath.fsum(e) + mpmath.exp(sg - m)
+        o = [mpmath.fsum(e[t] * mpmath.mpf(float(keys[t][d])) for t in range(len(keys))) / l
+             for d in range(d_v)]
+        outs.append([float(v) for v in o])
+        lses.append(float(m + mpmath.log(l)))
+    return np.array(outs), np.array(lses)
+
+
+def check_sink_brute_force(attend, seeds=range(4)):
+    """attend(..., sink) vs 50-digit brute force, including a sink that
+    dominates every score and a key set of one."""
+    for seed in seeds:
+        rng = np.random.default_rng(300 + seed)
+        d_qk = int(rng.integers(2, 9))
+        d_v = int(rng.integers(1, d_qk + 1))
+        T = int(rng.integers(1, 5))
+        R = 3
+        q = rng.standard_normal((R, d_qk)) * 2
+        k = rng.standard_normal((T, d_qk)) * 2
+        scale = float(rng.uniform(0.1, 1.5))
+        sink = np.array([rng.standard_normal(), 40.0, -3.0])
+        o, l = attend(q, k, scale, d_v, sink=sink)
+        eo, el = _mp_attend_sink(q.tolist(), k.tolist(), scale, d_v, sink)
+        _close(o, eo, 1e-13)
+        _close(l, el, 1e-13)
+
+
+def check_sink_single_token(attend):
+    """One key of score s and a sink sigma: out = v / (1 + e^(sigma - s)),
+    lse = ln(e^s + e^sigma) (closed form, computed here in 50 digits)."""
+    rng = np.random.default_rng(301)
+    d_qk, d_v = 576, 512
+    q = rng.standard_normal((2, d_qk))
+    k = rng.standard_normal((1, d_qk))
+    sink = np.array([0.3, -1.7])
+    o, l = attend(q, k, 1 / 24, d_v, sink=sink)
+    for r in range(2):
+        s = mpmath.mpf(1 / 24) * mpmath.fsum(mpmath.mpf(float(a)) * mpmath.mpf(float(b))
+                                            for a, b in zip(q[r], k[0]))
+        w = 1 / (1 + mpmath.exp(mpmath.mpf(float(sink[r])) - s))
+        _close(o[r], k[0, :d_v] * float(w), 1e-14)
+        _close(l[r], float(mpmath.log(mpmath.exp(s) + mpmath.exp(mpmath.mpf(float(sink[r]))))), 1e-14)
+
+
+def check_sink_as_extra_key(decode_dense):
+    """A per-head sink equals one more key whose value dims are zero and whose
+    RoPE dims give score sigma_h with every head's query: the same decode
+    without a sink over the longer key set. The key solves the h_q equations
+    scale * q_h[512:] . k_rope = sigma_h (h_q <= 64 unknowns, exact)."""
+    rng = np.random.default_rng(302)
+    d_qk, h_q, scale = 576, 5, 1 / 24
+    lens = [70, 1, 129]
+    cache, bt = _random_paged(rng, lens, d_qk, extra_pages=3)
+    sink = rng.standard_normal(h_q) + 1.0
+    q = rng.standard_normal((len(lens), 1, h_q, d_qk))
+    out, lse = decode_dense(q, cache, bt, np.array(lens), scale, False, sink=sink)
+    for b, L in enumerate(lens):
+        qb = q[b, 0]
+        k_rope, *_ = np.linalg.lstsq(scale * qb[:, 512:], sink, rcond=None)
+        extra = np.zeros(d_qk)
+        extra[512:] = k_rope
+        cb = cache.copy()
+        n = (L + PAGE - 1) // PAGE
+        bt_b = bt[b:b + 1].copy()
+        if L % PAGE == 0:                       # the extra key opens a fresh page
+            cb = np.concatenate([cb, np.zeros((1, PAGE, d_qk))])
+            bt_b = np.concatenate([bt_b, np.full((1, 1), -1)], axis=1)
+            bt_b[0, n] = cb.shape[0] - 1
+        page = bt_b[0, L // PAGE]
+        cb[page, L % PAGE] = extra
+        o2, l2 = decode_dense(q[b:b + 1], cb, bt_b, np.array([L + 1]), scale, False)
+        _close(out[b], o2[0], 1e-12)
+        _close(lse[b], l2[0], 1e-12)
+
+
+def check_sink_reductions(decode_dense, decode_sparse, attend, combine):
+    """sigma = -inf leaves every bit unchanged; an empty key set gives out 0
+    and lse = sigma; combining any split with the sink reproduces attend()
+    with the sink (the sink joins once, in the combine)."""
+    rng = np.random.default_rng(303)
+    d_qk, h_q = 576, 3
+    lens = [130, 0, 2]
+    cache, bt = _random_paged(rng, lens, d_qk, extra_pages=1)
+    q = rng.standard_normal((3, 2, h_q, d_qk))
+    o0, l0 = decode_dense(q, cache, bt, np.array(lens), 1 / 24, True)
+    o1, l1 = decode_dense(q, cache, bt, np.array(lens), 1 / 24, True, sink=np.full(h_q, -np.inf))
+    assert np.array_equal(o0, o1) and np.array_equal(l0, l1)
+    sink = np.array([0.5, -2.0, 7.0])
+    o2, l2 = decode_dense(q, cache, bt, np.array(lens), 1 / 24, True, sink=sink)
+    assert np.all(o2[1] == 0) and np.array_equal(l2[1, 0], sink) and np.array_equal(l2[1, 1], sink)
+    assert np.all(o2[2, 0] != 0)                     # causal row 0 of a 2-token request sees 1 key
+    idx = np.full((3, 2, 64), -1)
+    o3, l3 = decode_sparse(q, cache, bt, np.array(lens), idx, 1 / 24, sink=sink)
+    assert np.all(o3 == 0) and np.all(l3 == sink)
+    k = rng.standard_normal((200, d_qk))
+    qr = rng.standard_normal((h_q, d_qk))
+    o_ref, l_ref = attend(qr, k, 1 / 24, 512, sink=sink)
+    for cuts in ([0, 200], [0, 64, 64, 200], [0, 1, 199, 200]):
+        parts = [attend(qr, k[a:b], 1 / 24, 512) for a, b in zip(cuts[:-1], cuts[1:])]
+        o, l = combine(np.stack([p[0] for p in parts]), np.stack([p[1] for p in parts]), sink=sink)
+        _close(o, o_ref, 1e-13)
+        _close(l, l_ref, 1e-13)

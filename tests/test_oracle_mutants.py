@@ -147,3 +147,61 @@ def test_value_slice_mistake_caught():
         return out, lse
     assert _fails(C.check_single_token, decode_bad)
     assert _fails(C.check_golden_two_tokens, decode_bad)
+
+
+# ---------------------------------------------------------------- attention sink
+def _sink_negated(q, k, scale, d_v=512, sink=None):
+    return real_attend(q, k, scale, d_v, None if sink is None else -np.asarray(sink))
+
+
+def _sink_scaled(q, k, scale, d_v=512, sink=None):
+    return real_attend(q, k, scale, d_v, None if sink is None else scale * np.asarray(sink))
+
+
+def _sink_lse_dropped(q, k, scale, d_v=512, sink=None):
+    o, _ = real_attend(q, k, scale, d_v, sink)
+    _, l = real_attend(q, k, scale, d_v)
+    return o, l
+
+
+def _sink_out_dropped(q, k, scale, d_v=512, sink=None):
+    _, l = real_attend(q, k, scale, d_v, sink)
+    o, _ = real_attend(q, k, scale, d_v)
+    return o, l
+
+
+def _sink_carries_value(q, k, scale, d_v=512, sink=None):
+    """The sink key carries the first key's value instead of zero."""
+    o, l = real_attend(q, k, scale, d_v, sink)
+    k = np.asarray(k, float)
+    if sink is None or k.shape[0] == 0:
+        return o, l
+    w = np.exp(np.asarray(sink, float) - l)[:, None]
+    return o + w * k[0, :d_v], l
+
+
+SINK_MUTANTS = [_sink_negated, _sink_scaled, _sink_lse_dropped, _sink_out_dropped, _sink_carries_value]
+
+
+@pytest.mark.parametrize("mutant", SINK_MUTANTS, ids=lambda f: f.__name__)
+def test_sink_mutants_caught(mutant, monkeypatch):
+    caught = _fails(C.check_sink_brute_force, mutant)
+    caught = caught or _fails(C.check_sink_single_token, mutant)
+    monkeypatch.setattr(O, "attend", mutant)
+    caught = caught or _fails(C.check_sink_as_extra_key, O.decode_dense)
+    assert caught
+
+
+def test_sink_in_every_split_caught():
+    """A combine that adds the sink to each part instead of once."""
+    real_combine = O.combine
+
+    def per_part(o_parts, lse_parts, sink=None):
+        if sink is None:
+            return real_combine(o_parts, lse_parts)
+        lse_parts = np.asarray(lse_parts, float)
+        o_parts = np.asarray(o_parts, float)
+        lp = np.logaddexp(lse_parts, np.asarray(sink, float)[None, :])
+        op = o_parts * np.exp(lse_parts - lp)[..., None]
+        return real_combine(op, lp)
+    assert _fails(C.check_sink_reductions, O.decode_dense, O.decode_sparse, O.attend, per_part)

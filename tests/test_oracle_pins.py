@@ -60,3 +60,19 @@ def test_fp8_record_layout():
 
 def test_golden_two_tokens():
     C.check_golden_two_tokens(O.decode_dense)
+
+
+def test_sink_brute_force():
+    C.check_sink_brute_force(O.attend)
+
+
+def test_sink_single_token():
+    C.check_sink_single_token(O.attend)
+
+
+def test_sink_as_extra_key():
+    C.check_sink_as_extra_key(O.decode_dense)
+
+
+def test_sink_reductions():
+    C.check_sink_reductions(O.decode_dense, O.decode_sparse, O.attend, O.combine)

@@ -122,6 +122,7 @@ class DecodeInputs:
     cache_seqlens: torch.Tensor       # [B] int32
     indices: Optional[torch.Tensor] = None   # [B, s_q, topk] int32
     extra: dict = field(default_factory=dict)
+    sink: Optional[torch.Tensor] = None      # [h_q] fp32 per-head attention-sink logits
 
     @property
     def num_pages(self) -> int:
@@ -209,6 +210,19 @@ def make_inputs(w: Workload, *, poison_tail: bool = False, extra_pages: int = 0,
         extra={"pages_per_request": npages})
 
 
+def make_sink(h_q: int, seed: int) -> torch.Tensor:
+    """Per-head attention-sink logits [h_q] fp32, N(0, 1) + 1 (the scale of the
+    scores scale * q.k with unit-variance q and k), seeded."""
+    rng = np.random.Generator(np.random.PCG64(seed + 101))
+    return torch.from_numpy((rng.standard_normal(h_q) + 1.0).astype(np.float32))
+
+
+def with_sink(inp: "DecodeInputs", seed: int = 0) -> "DecodeInputs":
+    """The same inputs with seeded per-head sink logits attached."""
+    import dataclasses
+    return dataclasses.replace(inp, sink=make_sink(inp.workload.h_q, seed))
+
+
 def algorithmic_work(inp: DecodeInputs) -> dict:
     """FLOPs and bytes the method must do for one decode call.
 
@@ -271,4 +285,5 @@ def restrict(inp: DecodeInputs, requests) -> DecodeInputs:
     return DecodeInputs(
         workload=w, q=inp.q[requests].clone(), kcache=inp.kcache[pages].clone(),
         block_table=torch.from_numpy(new_bt), cache_seqlens=torch.tensor(sub_lens, dtype=torch.int32),
-        indices=None if inp.indices is None else inp.indices[requests].clone())
+        indices=None if inp.indices is None else inp.indices[requests].clone(),
+        sink=inp.sink)
