@@ -51,6 +51,7 @@ class MlaDecodeArgs(ctypes.Structure):
         ("num_pages", ctypes.c_int), ("block_table_stride", ctypes.c_int), ("num_sm_parts", ctypes.c_int),
         ("softmax_scale", ctypes.c_float), ("causal", ctypes.c_int), ("kv_format", ctypes.c_int),
         ("timeout_ns", ctypes.c_uint64), ("debug_flags", ctypes.c_uint32),
+        ("sink", ctypes.c_void_p),
     ]
 
 
@@ -83,6 +84,8 @@ def lib() -> ctypes.CDLL:
         L.mla_decode_sparse.argtypes = [ctypes.POINTER(MlaDecodeArgs), vp, i, vp]
         L.mla_combine.restype = i
         L.mla_combine.argtypes = [vp, sz, vp, i, i, i, vp, vp, vp]
+        L.mla_combine_sink.restype = i
+        L.mla_combine_sink.argtypes = [vp, sz, vp, i, i, i, i, vp, vp, vp, vp]
         L.mla_query_device_status.restype = i
         L.mla_query_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32), vp]
         L.mla_clear_device_status.restype = i
@@ -142,7 +145,7 @@ def mla_workspace_size(batch, s_q, h_q, h_kv, topk, num_sm_parts) -> int:
 def make_args(*, q, kcache, block_table, cache_seqlens, tile_md, num_splits, out, lse, workspace,
               batch, s_q, h_q, h_kv, num_pages, num_sm_parts, softmax_scale, causal, kv_format,
               block_table_stride=None, d_qk=576, d_v=512, page_size=64, timeout_ns=0, debug_flags=0,
-              workspace_bytes=None) -> MlaDecodeArgs:
+              workspace_bytes=None, sink=None) -> MlaDecodeArgs:
     a = MlaDecodeArgs()
     a.q, a.kcache, a.block_table = _ptr(q), _ptr(kcache), _ptr(block_table)
     a.cache_seqlens, a.tile_md, a.num_splits = _ptr(cache_seqlens), _ptr(tile_md), _ptr(num_splits)
@@ -158,6 +161,7 @@ def make_args(*, q, kcache, block_table, cache_seqlens, tile_md, num_splits, out
     a.kv_format = kv_format
     a.timeout_ns = timeout_ns
     a.debug_flags = debug_flags
+    a.sink = _ptr(sink)
     return a
 
 
@@ -181,6 +185,13 @@ def mla_combine(workspace, workspace_bytes, num_splits, num_units, rows_per_unit
                 stream=None):
     _check(lib().mla_combine(_ptr(workspace), workspace_bytes, _ptr(num_splits), num_units, rows_per_unit,
                              num_sm_parts, _ptr(out), _ptr(lse), _stream(stream)), "mla_combine")
+
+
+def mla_combine_sink(workspace, workspace_bytes, num_splits, num_units, rows_per_unit, num_sm_parts, h_q, sink,
+                     out, lse, stream=None):
+    _check(lib().mla_combine_sink(_ptr(workspace), workspace_bytes, _ptr(num_splits), num_units, rows_per_unit,
+                                  num_sm_parts, h_q, _ptr(sink), _ptr(out), _ptr(lse), _stream(stream)),
+           "mla_combine_sink")
 
 
 def mla_query_device_status(workspace, stream=None):

@@ -63,6 +63,7 @@ mla_status_t check_common(const mla_decode_args* a, int topk) {
   if (a->d_qk != kDqk || a->d_v != kDv || a->page_size != kPage) return MLA_ERR_INVALID_ARG;
   if (a->kv_format != MLA_KV_BF16 && a->kv_format != MLA_KV_FP8_E4M3) return MLA_ERR_INVALID_ARG;
   if (!(a->softmax_scale > 0.f) || !std::isfinite(a->softmax_scale)) return MLA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(a->sink) & 3u) != 0) return MLA_ERR_INVALID_ARG;
   if (a->h_kv != 1) return MLA_ERR_UNSUPPORTED;
   const int rows = rows_of(a->s_q, a->h_q, a->h_kv, topk);
   if (rows > MLA_MAX_ROWS) return MLA_ERR_UNSUPPORTED;
@@ -118,12 +119,14 @@ mla_status_t run_decode(const mla_decode_args* a, const int32_t* indices, int to
   p.status = reinterpret_cast<uint32_t*>(ws);
   p.timeout_ns = a->timeout_ns ? a->timeout_ns : 2000000000ull;
   p.debug_flags = a->debug_flags;
+  p.sink = a->sink;
   const int rows_per_cta = rows < kRowsPerCta ? rows : kRowsPerCta;
   const cudaError_t e = pair ? launch_decode_pair(tq, tkv, p, a->num_sm_parts, mode == kModeSparse, stream)
                              : launch_decode(rows_per_cta, mode, tq, tkv, p, a->num_sm_parts, row_groups, stream);
   if (e != cudaSuccess) return MLA_ERR_CUDA;
   if (a->debug_flags & MLA_DEBUG_SKIP_COMBINE) return MLA_OK;
-  return launch_combine(a->workspace, U, rows, a->num_sm_parts, a->num_splits, a->out, a->lse, stream);
+  return launch_combine(a->workspace, U, rows, a->num_sm_parts, a->num_splits, a->h_q, a->sink, a->out, a->lse,
+                        stream);
 }
 
 }  // namespace
@@ -196,15 +199,24 @@ mla_status_t mla_decode_sparse(const mla_decode_args* args, const int32_t* indic
   return run_decode(args, indices, topk, reinterpret_cast<cudaStream_t>(stream));
 }
 
-mla_status_t mla_combine(const void* workspace, size_t workspace_bytes, const int32_t* num_splits, int num_units,
-                         int rows_per_unit, int num_sm_parts, void* out, float* lse, mla_stream_t stream) {
+mla_status_t mla_combine_sink(const void* workspace, size_t workspace_bytes, const int32_t* num_splits,
+                              int num_units, int rows_per_unit, int num_sm_parts, int h_q, const float* sink,
+                              void* out, float* lse, mla_stream_t stream) {
   if (!workspace || !num_splits || !out || !lse || num_units <= 0 || rows_per_unit <= 0 || num_sm_parts <= 0)
     return MLA_ERR_INVALID_ARG;
   if (!aligned16(out) || !aligned16(workspace)) return MLA_ERR_INVALID_ARG;
+  if (sink && (h_q <= 0 || rows_per_unit % h_q != 0 || (reinterpret_cast<uintptr_t>(sink) & 3u) != 0))
+    return MLA_ERR_INVALID_ARG;
   if (workspace_bytes < ws_layout(num_units, rows_per_unit, num_sm_parts).total)
     return MLA_ERR_WORKSPACE_TOO_SMALL;
-  return launch_combine(workspace, num_units, rows_per_unit, num_sm_parts, num_splits, out, lse,
-                        reinterpret_cast<cudaStream_t>(stream));
+  return launch_combine(workspace, num_units, rows_per_unit, num_sm_parts, num_splits, sink ? h_q : 1, sink, out,
+                        lse, reinterpret_cast<cudaStream_t>(stream));
+}
+
+mla_status_t mla_combine(const void* workspace, size_t workspace_bytes, const int32_t* num_splits, int num_units,
+                         int rows_per_unit, int num_sm_parts, void* out, float* lse, mla_stream_t stream) {
+  return mla_combine_sink(workspace, workspace_bytes, num_splits, num_units, rows_per_unit, num_sm_parts, 1,
+                          nullptr, out, lse, stream);
 }
 
 mla_status_t mla_query_device_status(const void* workspace, uint32_t* status_bits, mla_stream_t stream) {

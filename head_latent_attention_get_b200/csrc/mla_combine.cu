@@ -3,6 +3,10 @@
 // one request's KV). Each split s of a unit holds its own softmax-normalised
 // partial output o_s and log-sum-exp lse_s over a disjoint subset of the keys:
 //   lse = ln sum_s exp(lse_s),   out = sum_s exp(lse_s - lse) * o_s.
+// With a per-head attention sink sigma (an extra logit with a zero value,
+// "[flashinfer] ...", section 2), it joins here once per row, after the
+// splits: lse' = ln(e^lse + e^sigma), out *= e^(lse - lse'); a unit with no
+// split at all gets out 0 and lse sigma.
 // One block per (unit, chunk of 4 rows); a unit that was not split (its
 // piece wrote the output directly) costs the block one read. Each half-block
 // of 128 threads merges one row at a time, each thread owning 4 of the 512
@@ -19,7 +23,7 @@ constexpr int kCombineRows = 4;  // rows per block
 
 __global__ void __launch_bounds__(kCombineThreads) mla_combine_kernel(
     const float* __restrict__ part_lse, const float* __restrict__ part_o, const int32_t* __restrict__ split_ptr,
-    int rows, __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
+    int rows, int h_q, const float* __restrict__ sink, __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
   const int half = threadIdx.x >> 7;
   const int d = (threadIdx.x & 127) * 4;
   const int u = blockIdx.x;
@@ -45,6 +49,10 @@ __global__ void __launch_bounds__(kCombineThreads) mla_combine_kernel(
           }
         }
       }
+      if (sink != nullptr) {
+        const float f = fold_sink(L, sink[r % h_q]);
+        acc.x *= f; acc.y *= f; acc.z *= f; acc.w *= f;
+      }
       __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
       __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
       uint2 packed;
@@ -57,13 +65,13 @@ __global__ void __launch_bounds__(kCombineThreads) mla_combine_kernel(
 }
 
 mla_status_t launch_combine(const void* workspace, int units, int rows, int parts, const int32_t* split_ptr,
-                            void* out, float* lse, cudaStream_t stream) {
+                            int h_q, const float* sink, void* out, float* lse, cudaStream_t stream) {
   const WsLayout w = ws_layout(units, rows, parts);
   const char* ws = static_cast<const char*>(workspace);
   const dim3 grid(units, (rows + kCombineRows - 1) / kCombineRows);
   mla_combine_kernel<<<grid, kCombineThreads, 0, stream>>>(
-      reinterpret_cast<const float*>(ws + w.lse_off), reinterpret_cast<const float*>(ws + w.o_off), split_ptr, rows,
-      static_cast<__nv_bfloat16*>(out), lse);
+      reinterpret_cast<const float*>(ws + w.lse_off), reinterpret_cast<const float*>(ws + w.o_off), split_ptr, rows, h_q,
+      sink, static_cast<__nv_bfloat16*>(out), lse);
   return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 

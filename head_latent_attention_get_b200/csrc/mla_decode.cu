@@ -636,6 +636,7 @@ __global__ void __launch_bounds__(MODE == kModeBf16 ? 256 : 256 + 2 * kGatherThr
           inv = 1.f / l_sum;
           lse = m_used * p.scale + logf(l_sum);
         }
+        if (pc.single && rvalid && p.sink != nullptr) inv *= fold_sink(lse, p.sink[(row0 + r) % p.h_q]);
         c->inv_l[r] = inv;
         if (rvalid) {
           const size_t grow_all = (size_t)pc.unit * p.rows + row0 + r;

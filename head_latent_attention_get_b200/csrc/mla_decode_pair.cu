@@ -632,6 +632,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SPARSE ? kThreadsSpa
         inv = 1.f / l_tot;
         lse = m_used * p.scale + logf(l_tot);
       }
+      if (pc.single && rvalid && p.sink != nullptr) inv *= fold_sink(lse, p.sink[grow % p.h_q]);
       const size_t orow = (size_t)pc.unit * p.rows + grow;
       if (rvalid && half == 0) {
         if (pc.single) p.lse[orow] = lse;

@@ -27,7 +27,28 @@ struct DecodeParams {
   uint32_t* status;                         // device status word
   uint64_t timeout_ns;
   uint32_t debug_flags;
+  const float* sink;                        // per-head sink logits [h_q], or null
 };
+
+#ifdef __CUDACC__
+// Attention sink ("[flashinfer] ...", section 2: an optional per-head sink,
+// sinks [num_heads] float32): one more logit sigma per head that joins the
+// softmax denominator with a zero value vector. Folded into a finished
+// softmax with log-sum-exp `lse` (-inf for an empty key set):
+//   L = ln(e^lse + e^sigma),  out *= e^(lse - L),  lse = L.
+// Returns the factor on the output and replaces lse by L; written with
+// max + log1p so that no exponential overflows.
+__device__ __forceinline__ float fold_sink(float& lse, float sigma) {
+  if (lse == -INFINITY) {
+    lse = sigma;
+    return 0.f;
+  }
+  const float L = fmaxf(lse, sigma) + log1pf(expf(-fabsf(lse - sigma)));
+  const float f = expf(lse - L);
+  lse = L;
+  return f;
+}
+#endif
 
 cudaError_t launch_decode(int rows_per_cta, int mode, const CUtensorMap& tq, const CUtensorMap& tkv,
                           const DecodeParams& p, int parts, int row_groups, cudaStream_t stream);
@@ -39,7 +60,8 @@ cudaError_t launch_decode_pair(const CUtensorMap& tq, const CUtensorMap& tkv, co
 int max_pair_clusters();
 mla_status_t launch_metadata(const int32_t* seqlens, int U, int topk, int parts, int32_t* tile_md,
                              int32_t* num_splits, cudaStream_t stream);
+// `sink` (device fp32 [h_q] or null): the head of row r of a unit is r % h_q.
 mla_status_t launch_combine(const void* workspace, int units, int rows, int parts, const int32_t* split_ptr,
-                            void* out, float* lse, cudaStream_t stream);
+                            int h_q, const float* sink, void* out, float* lse, cudaStream_t stream);
 
 }  // namespace mla

@@ -15,7 +15,7 @@ from . import _capi as C
 
 class DecodeRunner:
     def __init__(self, q, kcache, block_table, cache_seqlens, *, softmax_scale, causal=False,
-                 indices=None, num_sm_parts=None, timeout_ns=0, debug_flags=0):
+                 indices=None, num_sm_parts=None, timeout_ns=0, debug_flags=0, sink=None):
         dev = q.device
         assert dev.type == "cuda", "the decode path runs on a CUDA device only"
         self.batch, self.s_q, self.h_q, d = q.shape
@@ -33,12 +33,17 @@ class DecodeRunner:
         self.lse = torch.empty(self.batch, self.s_q, self.h_q, dtype=torch.float32, device=dev)
         self.q, self.kcache, self.block_table, self.cache_seqlens = q, kcache, block_table, cache_seqlens
         self.indices = indices
+        if sink is not None:
+            assert sink.device == dev and sink.dtype == torch.float32 and sink.shape == (self.h_q,)
+            sink = sink.contiguous()
+        self.sink = sink
         self.args = C.make_args(
             q=q, kcache=kcache, block_table=block_table, cache_seqlens=cache_seqlens,
             tile_md=self.tile_md, num_splits=self.num_splits, out=self.out, lse=self.lse,
             workspace=self.workspace, batch=self.batch, s_q=self.s_q, h_q=self.h_q, h_kv=1,
             num_pages=kcache.shape[0], num_sm_parts=self.parts, softmax_scale=softmax_scale,
-            causal=causal, kv_format=self.kv_format, timeout_ns=timeout_ns, debug_flags=debug_flags)
+            causal=causal, kv_format=self.kv_format, timeout_ns=timeout_ns, debug_flags=debug_flags,
+            sink=sink)
 
     def plan(self, stream=None):
         C.mla_get_metadata(self.cache_seqlens, self.batch, self.s_q, self.h_q, 1, self.topk, self.parts,

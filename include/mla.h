@@ -179,6 +179,16 @@ typedef struct {
   int kv_format;                /* MLA_KV_BF16 or MLA_KV_FP8_E4M3 */
   uint64_t timeout_ns;          /* limit of every device wait; 0 = 2 s */
   uint32_t debug_flags;         /* MLA_DEBUG_* test hooks; 0 normally */
+  const float* sink;            /* device fp32 [h_q], 4-B aligned, or NULL: per-head
+                                   attention-sink logits (FlashInfer page, section 2,
+                                   "sinks [num_heads] float32"). sink[h] joins the
+                                   softmax denominator of every row of head h as one
+                                   more logit, in the units of softmax_scale * q.k,
+                                   whose value vector is zero:
+                                     lse = ln(sum_t e^(s_t) + e^sink[h]),
+                                     out = sum_t e^(s_t - lse) v_t.
+                                   An empty key set then gives out 0, lse = sink[h];
+                                   sink[h] = -inf is the same as no sink. */
 } mla_decode_args;
 
 /* Paged decoding: enqueues the decode kernel and the split combine.
@@ -234,6 +244,19 @@ mla_status_t mla_decode_sparse(const mla_decode_args* args, const int32_t* indic
 mla_status_t mla_combine(const void* workspace, size_t workspace_bytes, const int32_t* num_splits,
                          int num_units, int rows_per_unit, int num_sm_parts, void* out, float* lse,
                          mla_stream_t stream);
+
+/* mla_combine with a per-head attention sink (see mla_decode_args.sink):
+ * after the splits are merged, row r of a unit (head r % h_q) takes
+ *   lse' = ln(e^lse + e^sink[r % h_q]),  out *= e^(lse - lse'),
+ * and a unit with n == 0 gets out = 0, lse = sink[r % h_q]. Units with
+ * n == 1 are left alone (their decode piece folded the sink in already).
+ * sink: device fp32 [h_q], 4-B aligned, or NULL (then identical to
+ * mla_combine and h_q is ignored). Errors as mla_combine; INVALID_ARG also
+ * when sink is given and h_q <= 0, rows_per_unit % h_q != 0 or sink is
+ * misaligned. */
+mla_status_t mla_combine_sink(const void* workspace, size_t workspace_bytes, const int32_t* num_splits,
+                              int num_units, int rows_per_unit, int num_sm_parts, int h_q, const float* sink,
+                              void* out, float* lse, mla_stream_t stream);
 
 /* Reads the device status word (blocks until `stream` reaches this point).
  * Returns MLA_OK, MLA_ERR_DEVICE_TIMEOUT or MLA_ERR_DEVICE_BOUNDS (timeout

@@ -79,6 +79,7 @@ def _fake_args(**over):
     (dict(h_q=256), C.MLA_ERR_UNSUPPORTED),
     (dict(s_q=2, h_q=128), C.MLA_ERR_UNSUPPORTED),
     (dict(workspace_bytes=1024), C.MLA_ERR_WORKSPACE_TOO_SMALL),
+    (dict(sink=0x300002), C.MLA_ERR_INVALID_ARG),             # misaligned sink
 ])
 def test_decode_rejects_bad_arguments(over, code):
     a = _fake_args(**over)
@@ -102,6 +103,11 @@ def test_metadata_rejects_bad_arguments():
     assert L.mla_get_metadata(None, 2, 1, 16, 1, 0, 8, 0x2000, 0x3000, None) == C.MLA_ERR_INVALID_ARG
     assert L.mla_get_metadata(0x1000, 2, 1, 16, 2, 0, 8, 0x2000, 0x3000, None) == C.MLA_ERR_UNSUPPORTED
     assert L.mla_combine(None, 0, None, 1, 1, 1, None, None, None) == C.MLA_ERR_INVALID_ARG
+    ws, ns, out, lse, sink = 0x100000, 0x200000, 0x300000, 0x400000, 0x500000
+    big = 1 << 40
+    for h_q, sk in ((0, sink), (3, sink), (16, sink + 2)):   # h_q <= 0, rows % h_q, misaligned
+        assert L.mla_combine_sink(ws, big, ns, 4, 32, 8, h_q, sk, out, lse, None) == C.MLA_ERR_INVALID_ARG
+    assert L.mla_combine_sink(ws, 1024, ns, 4, 32, 8, 16, sink, out, lse, None) == C.MLA_ERR_WORKSPACE_TOO_SMALL
     assert L.mla_query_device_status(None, None, None) == C.MLA_ERR_INVALID_ARG
 
 
@@ -144,3 +150,20 @@ def test_host_scheduler_random_and_mtp():
     md, ns = host_schedule(w.seqlens, w.batch, 2, 16, 0, 148)
     info = S.check_schedule(md, ns, w.seqlens, w.batch, 2, 0, 148)
     assert info["splits"] <= w.batch + 148
+
+
+def test_args_struct_layout_matches_header(tmp_path):
+    """The ctypes mirror of mla_decode_args has the C compiler's size and
+    field offsets (gcc on the header itself)."""
+    fields = [f for f, _ in C.MlaDecodeArgs._fields_]
+    src = tmp_path / "layout.c"
+    src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "mla.h"\nint main(void) {\n'
+                   '  printf("%zu\\n", sizeof(mla_decode_args));\n'
+                   + "".join(f'  printf("%zu\\n", offsetof(mla_decode_args, {f}));\n' for f in fields)
+                   + "  return 0;\n}\n")
+    exe = tmp_path / "layout"
+    import subprocess
+    subprocess.run(["gcc", "-std=c99", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    got = [int(x) for x in subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()]
+    assert got[0] == ctypes.sizeof(C.MlaDecodeArgs)
+    assert got[1:] == [getattr(C.MlaDecodeArgs, f).offset for f in fields]
