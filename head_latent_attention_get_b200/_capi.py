@@ -68,6 +68,8 @@ def lib() -> ctypes.CDLL:
         i, vp, sz = ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t
         L.mla_status_string.restype = ctypes.c_char_p
         L.mla_status_string.argtypes = [i]
+        L.mla_decode_geometry.restype = i
+        L.mla_decode_geometry.argtypes = [i, i, i, i, ctypes.POINTER(i), ctypes.POINTER(i)]
         L.mla_get_num_sm_parts.restype = i
         L.mla_get_num_sm_parts.argtypes = [i, i, i, i, i, ctypes.POINTER(i)]
         L.mla_get_metadata.restype = i
@@ -118,6 +120,14 @@ def _check(code: int, where: str):
 
 def mla_status_string(code: int) -> str:
     return lib().mla_status_string(code).decode()
+
+
+def mla_decode_geometry(s_q: int, h_q: int, h_kv: int = 1, topk: int = 0):
+    """(units per request, rows per unit) of a decode problem."""
+    upr, rows = ctypes.c_int(0), ctypes.c_int(0)
+    _check(lib().mla_decode_geometry(s_q, h_q, h_kv, topk, ctypes.byref(upr), ctypes.byref(rows)),
+           "mla_decode_geometry")
+    return upr.value, rows.value
 
 
 def mla_get_num_sm_parts(device: int, s_q: int, h_q: int, h_kv: int = 1, topk: int = 0) -> int:

@@ -47,8 +47,12 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-int units_of(int batch, int s_q, int topk) { return topk > 0 ? batch * s_q : batch; }
-int rows_of(int s_q, int h_q, int h_kv, int topk) { return topk > 0 ? h_q / h_kv : s_q * h_q / h_kv; }
+// {units per request, rows per unit}; rows 0 when the sizes are out of range.
+Geometry geometry_of(int s_q, int h_q, int h_kv, int topk) {
+  Geometry g{0, 0};
+  if (!unit_geometry(s_q, h_q, h_kv, topk, &g)) g = Geometry{0, 0};
+  return g;
+}
 
 mla_status_t check_common(const mla_decode_args* a, int topk) {
   if (!a) return MLA_ERR_INVALID_ARG;
@@ -65,9 +69,11 @@ mla_status_t check_common(const mla_decode_args* a, int topk) {
   if (!(a->softmax_scale > 0.f) || !std::isfinite(a->softmax_scale)) return MLA_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(a->sink) & 3u) != 0) return MLA_ERR_INVALID_ARG;
   if (a->h_kv != 1) return MLA_ERR_UNSUPPORTED;
-  const int rows = rows_of(a->s_q, a->h_q, a->h_kv, topk);
-  if (rows > MLA_MAX_ROWS) return MLA_ERR_UNSUPPORTED;
-  const int U = units_of(a->batch, a->s_q, topk);
+  const Geometry g = geometry_of(a->s_q, a->h_q, a->h_kv, topk);
+  const int rows = g.rows;
+  if (rows <= 0 || rows > MLA_MAX_ROWS) return MLA_ERR_UNSUPPORTED;
+  if ((long long)a->batch * g.units_per_req > 0x7fffffff) return MLA_ERR_UNSUPPORTED;
+  const int U = a->batch * g.units_per_req;
   if (a->workspace_bytes < ws_layout(U, rows, a->num_sm_parts).total) return MLA_ERR_WORKSPACE_TOO_SMALL;
   if ((size_t)U * rows > (size_t)0x7fffffff / kDqk || (size_t)a->num_pages * kPage > 0x7fffffffu)
     return MLA_ERR_UNSUPPORTED;
@@ -75,8 +81,9 @@ mla_status_t check_common(const mla_decode_args* a, int topk) {
 }
 
 mla_status_t run_decode(const mla_decode_args* a, const int32_t* indices, int topk, cudaStream_t stream) {
-  const int rows = rows_of(a->s_q, a->h_q, a->h_kv, topk);
-  const int U = units_of(a->batch, a->s_q, topk);
+  const Geometry g = geometry_of(a->s_q, a->h_q, a->h_kv, topk);
+  const int rows = g.rows;
+  const int U = a->batch * g.units_per_req;
   const int mode = topk > 0 ? kModeSparse : (a->kv_format == MLA_KV_FP8_E4M3 ? kModeFp8 : kModeBf16);
   // Q rows of every unit, and (bf16 paged cache only) the cache as
   // [pages*64 tokens][576 dims]; boxes of 64 x 64 with 128-B swizzle. The FP8
@@ -97,6 +104,7 @@ mla_status_t run_decode(const mla_decode_args* a, const int32_t* indices, int to
   std::memset(&p, 0, sizeof(p));
   p.units = U;
   p.rows = rows;
+  p.upr = g.units_per_req;
   p.h_q = a->h_q;
   p.s_q = a->s_q;
   p.causal = (topk == 0 && a->causal) ? 1 : 0;
@@ -149,8 +157,8 @@ const char* mla_status_string(mla_status_t s) {
 mla_status_t mla_get_num_sm_parts(int device, int s_q, int h_q, int h_kv, int topk, int* num_sm_parts) {
   if (!num_sm_parts || s_q <= 0 || h_q <= 0 || h_kv <= 0 || topk < 0) return MLA_ERR_INVALID_ARG;
   if (h_kv != 1) return MLA_ERR_UNSUPPORTED;
-  const int rows = rows_of(s_q, h_q, h_kv, topk);
-  if (rows > MLA_MAX_ROWS) return MLA_ERR_UNSUPPORTED;
+  const int rows = geometry_of(s_q, h_q, h_kv, topk).rows;
+  if (rows <= 0 || rows > MLA_MAX_ROWS) return MLA_ERR_UNSUPPORTED;
   int sms = 0;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || sms <= 0)
     return MLA_ERR_CUDA;
@@ -175,13 +183,29 @@ mla_status_t mla_get_metadata(const int32_t* cache_seqlens, int batch, int s_q, 
   if (topk < 0 || (topk > 0 && topk % 64 != 0)) return MLA_ERR_INVALID_ARG;
   if (topk == 0 && !cache_seqlens) return MLA_ERR_INVALID_ARG;
   if (h_kv != 1) return MLA_ERR_UNSUPPORTED;
-  return launch_metadata(cache_seqlens, units_of(batch, s_q, topk), topk, num_sm_parts, tile_md, num_splits,
-                         reinterpret_cast<cudaStream_t>(stream));
+  const Geometry g = geometry_of(s_q, h_q, h_kv, topk);
+  if (g.rows <= 0 || (long long)batch * g.units_per_req > 0x7fffffff) return MLA_ERR_UNSUPPORTED;
+  return launch_metadata(cache_seqlens, batch * g.units_per_req, g.units_per_req, topk, num_sm_parts, tile_md,
+                         num_splits, reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t mla_workspace_size(int batch, int s_q, int h_q, int h_kv, int topk, int num_sm_parts) {
   if (batch <= 0 || s_q <= 0 || h_q <= 0 || h_kv <= 0 || topk < 0 || num_sm_parts <= 0) return 0;
-  return ws_layout(units_of(batch, s_q, topk), rows_of(s_q, h_q, h_kv, topk), num_sm_parts).total;
+  const Geometry g = geometry_of(s_q, h_q, h_kv, topk);
+  if (g.rows <= 0 || (long long)batch * g.units_per_req > 0x7fffffff) return 0;
+  return ws_layout(batch * g.units_per_req, g.rows, num_sm_parts).total;
+}
+
+mla_status_t mla_decode_geometry(int s_q, int h_q, int h_kv, int topk, int* units_per_request,
+                                 int* rows_per_unit) {
+  if (!units_per_request || !rows_per_unit || s_q <= 0 || h_q <= 0 || h_kv <= 0 || topk < 0)
+    return MLA_ERR_INVALID_ARG;
+  if (h_kv != 1) return MLA_ERR_UNSUPPORTED;
+  const Geometry g = geometry_of(s_q, h_q, h_kv, topk);
+  if (g.rows <= 0 || g.rows > MLA_MAX_ROWS) return MLA_ERR_UNSUPPORTED;
+  *units_per_request = g.units_per_req;
+  *rows_per_unit = g.rows;
+  return MLA_OK;
 }
 
 mla_status_t mla_decode_paged(const mla_decode_args* args, mla_stream_t stream) {
@@ -205,7 +229,7 @@ mla_status_t mla_combine_sink(const void* workspace, size_t workspace_bytes, con
   if (!workspace || !num_splits || !out || !lse || num_units <= 0 || rows_per_unit <= 0 || num_sm_parts <= 0)
     return MLA_ERR_INVALID_ARG;
   if (!aligned16(out) || !aligned16(workspace)) return MLA_ERR_INVALID_ARG;
-  if (sink && (h_q <= 0 || rows_per_unit % h_q != 0 || (reinterpret_cast<uintptr_t>(sink) & 3u) != 0))
+  if (sink && (h_q <= 0 || (reinterpret_cast<uintptr_t>(sink) & 3u) != 0))
     return MLA_ERR_INVALID_ARG;
   if (workspace_bytes < ws_layout(num_units, rows_per_unit, num_sm_parts).total)
     return MLA_ERR_WORKSPACE_TOO_SMALL;

@@ -50,7 +50,7 @@ __global__ void __launch_bounds__(kCombineThreads) mla_combine_kernel(
         }
       }
       if (sink != nullptr) {
-        const float f = fold_sink(L, sink[r % h_q]);
+        const float f = fold_sink(L, sink[(int)(orow % h_q)]);
         acc.x *= f; acc.y *= f; acc.z *= f; acc.w *= f;
       }
       __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);

@@ -32,6 +32,32 @@ __host__ __device__ inline WsLayout ws_layout(int units, int rows, int num_parts
   return w;
 }
 
+// Work-unit geometry. Sparse decoding has one unit per (request, query
+// token) of h_q/h_kv rows (at most MLA_MAX_ROWS). Paged decoding cuts the
+// R = s_q*h_q/h_kv query rows of a request into the fewest equal blocks of at
+// most MLA_MAX_ROWS rows (the smallest count >= ceil(R/128) that divides R);
+// each block is a unit, and the units of a request are consecutive, so unit u
+// covers rows [u*rows, (u+1)*rows) of the flattened [batch*s_q*h_q] row axis
+// and belongs to request u / units_per_req. Returns false for sizes out of
+// range (R above 2^20 rows).
+struct Geometry {
+  int units_per_req, rows;
+};
+__host__ __device__ inline bool unit_geometry(int s_q, int h_q, int h_kv, int topk, Geometry* g) {
+  if (s_q <= 0 || h_q <= 0 || h_kv <= 0 || (long long)s_q * h_q > (1 << 20)) return false;
+  if (topk > 0) {
+    g->units_per_req = s_q;
+    g->rows = h_q / h_kv;
+    return true;
+  }
+  const int R = s_q * h_q / h_kv;
+  int n = (R + MLA_MAX_ROWS - 1) / MLA_MAX_ROWS;
+  while (R % n != 0) ++n;
+  g->units_per_req = n;
+  g->rows = R / n;
+  return true;
+}
+
 // Scheduler part descriptor, MLA_TILE_MD_INTS int32 per part.
 struct PartMd {
   int32_t begin_unit, begin_tile, end_unit, end_tile, first_ws_idx, payload, pad0, pad1;

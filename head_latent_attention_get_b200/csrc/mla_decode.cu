@@ -336,7 +336,7 @@ __global__ void __launch_bounds__(MODE == kModeBf16 ? 256 : 256 + 2 * kGatherThr
           ++q_issued;
         }
         if (MODE == kModeBf16 && !stop) {
-          const int req = pc.unit;
+          const int req = unit_req(p, pc.unit);
           const int npg = (p.seqlens[req] + kPage - 1) / kPage;
           for (int k = pc.t0; k < pc.t1 && !stop; ++k) {
             int pa = page_of(p, req, 2 * k, npg);
@@ -367,7 +367,7 @@ __global__ void __launch_bounds__(MODE == kModeBf16 ? 256 : 256 + 2 * kGatherThr
       int vc = 0;
       bool stop = false;
       while (!stop && it.next(pc)) {
-        const int req = pc.unit;
+        const int req = unit_req(p, pc.unit);
         const int npg = (p.seqlens[req] + kPage - 1) / kPage;
         for (int k = pc.t0; k < pc.t1 && !stop; ++k) {
           int pg[2];
@@ -507,7 +507,7 @@ __global__ void __launch_bounds__(MODE == kModeBf16 ? 256 : 256 + 2 * kGatherThr
       if (MODE != kModeSparse) {
         const int Ls = p.seqlens[req];
         limit = Ls;
-        if (p.causal) limit = Ls - p.s_q + grow / p.h_q + 1;
+        if (p.causal) limit = Ls - p.s_q + row_query(p, pc.unit, grow) + 1;
       }
       float m_used = -INFINITY, l_sum = 0.f;
       int last_gt = -1;
@@ -636,7 +636,7 @@ __global__ void __launch_bounds__(MODE == kModeBf16 ? 256 : 256 + 2 * kGatherThr
           inv = 1.f / l_sum;
           lse = m_used * p.scale + logf(l_sum);
         }
-        if (pc.single && rvalid && p.sink != nullptr) inv *= fold_sink(lse, p.sink[(row0 + r) % p.h_q]);
+        if (pc.single && rvalid && p.sink != nullptr) inv *= fold_sink(lse, p.sink[row_head(p, pc.unit, row0 + r)]);
         c->inv_l[r] = inv;
         if (rvalid) {
           const size_t grow_all = (size_t)pc.unit * p.rows + row0 + r;

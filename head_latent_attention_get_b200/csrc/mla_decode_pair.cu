@@ -518,7 +518,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SPARSE ? kThreadsSpa
     while (!stop && it.next(pc)) {
       const int req = unit_req(p, pc.unit);
       const int Ls = p.seqlens[req];
-      const int limit = p.causal ? Ls - p.s_q + grow / p.h_q + 1 : Ls;
+      const int limit = p.causal ? Ls - p.s_q + row_query(p, pc.unit, grow) + 1 : Ls;
       float m_used = -INFINITY, l_sum = 0.f;
       int last_gt = -1;
       for (int k = pc.t0; k < pc.t1 && !stop; k += 2, ++gt) {
@@ -632,7 +632,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SPARSE ? kThreadsSpa
         inv = 1.f / l_tot;
         lse = m_used * p.scale + logf(l_tot);
       }
-      if (pc.single && rvalid && p.sink != nullptr) inv *= fold_sink(lse, p.sink[grow % p.h_q]);
+      if (pc.single && rvalid && p.sink != nullptr) inv *= fold_sink(lse, p.sink[row_head(p, pc.unit, grow)]);
       const size_t orow = (size_t)pc.unit * p.rows + grow;
       if (rvalid && half == 0) {
         if (pc.single) p.lse[orow] = lse;

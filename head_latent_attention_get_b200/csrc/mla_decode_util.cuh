@@ -29,7 +29,7 @@ struct PieceIter {
   }
   __device__ int tiles_of(int unit) const {
     if (p->topk > 0) return (p->topk + kTile - 1) / kTile;
-    int L = p->seqlens[unit];
+    int L = p->seqlens[unit / p->upr];
     return L > 0 ? (L + kTile - 1) / kTile : 0;
   }
   __device__ bool next(Piece& pc) {
@@ -103,8 +103,17 @@ __device__ __forceinline__ int sparse_row(const DecodeParams& p, int unit, int s
   return pg * kPage + (idx % kPage);
 }
 
-__device__ __forceinline__ int unit_req(const DecodeParams& p, int unit) {
-  return p.topk > 0 ? unit / p.s_q : unit;
+__device__ __forceinline__ int unit_req(const DecodeParams& p, int unit) { return unit / p.upr; }
+
+// Query token index (0..s_q-1) of row r of a unit: rows are laid out
+// [request][query token][head] on one flattened axis.
+__device__ __forceinline__ int row_query(const DecodeParams& p, int unit, int r) {
+  return ((unit * p.rows + r) / p.h_q) % p.s_q;
+}
+
+// Head of row r of a unit (the index into the per-head sink).
+__device__ __forceinline__ int row_head(const DecodeParams& p, int unit, int r) {
+  return (unit * p.rows + r) % p.h_q;
 }
 
 // Number of valid keys of tile k for a row limit (dense): tokens [128k, 128k+128).

@@ -11,6 +11,7 @@ enum KvMode : int { kModeBf16 = 0, kModeFp8 = 1, kModeSparse = 2 };
 
 struct DecodeParams {
   int units, rows, h_q, s_q, causal, topk;  // rows = query rows per unit
+  int upr;                                  // units per request (unit u -> request u / upr)
   float scale, scale_log2;                  // softmax scale, and scale * log2(e)
   int num_pages, bt_stride;
   const int32_t* block_table;
@@ -58,7 +59,8 @@ cudaError_t launch_decode_pair(const CUtensorMap& tq, const CUtensorMap& tkv, co
                                bool sparse, cudaStream_t stream);
 // How many CTA pairs of the pair kernel can be resident at once on the current device (0 if unknown).
 int max_pair_clusters();
-mla_status_t launch_metadata(const int32_t* seqlens, int U, int topk, int parts, int32_t* tile_md,
+// Unit u reads seqlens[u / upr] (paged decoding; upr = units per request).
+mla_status_t launch_metadata(const int32_t* seqlens, int U, int upr, int topk, int parts, int32_t* tile_md,
                              int32_t* num_splits, cudaStream_t stream);
 // `sink` (device fp32 [h_q] or null): the head of row r of a unit is r % h_q.
 mla_status_t launch_combine(const void* workspace, int units, int rows, int parts, const int32_t* split_ptr,

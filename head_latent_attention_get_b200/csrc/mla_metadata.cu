@@ -2,8 +2,8 @@
 // section "Obtenir les métadonnées MLA" — computed once per decode step from
 // cache_seqlens and reused by every layer).
 //
-// Every work unit (a request for paged decoding, a (request, query token)
-// pair for sparse decoding) costs n_u tiles of 128 tokens plus a fixed
+// Every work unit (a block of at most 128 query rows of a request for paged
+// decoding, a (request, query token) pair for sparse decoding) costs n_u tiles of 128 tokens plus a fixed
 // overhead of kSchedOverhead tiles (loading Q, writing a partial result,
 // combining). Units are laid end to end on a cost axis [0, total); part p
 // takes the cost range [p*payload, (p+1)*payload) with payload =
@@ -24,9 +24,9 @@
 
 namespace mla {
 
-__host__ __device__ inline int unit_tiles(const int32_t* seqlens, int u, int topk) {
+__host__ __device__ inline int unit_tiles(const int32_t* seqlens, int u, int upr, int topk) {
   if (topk > 0) return (topk + kTile - 1) / kTile;
-  int L = seqlens[u];
+  int L = seqlens[u / upr];
   return L > 0 ? (L + kTile - 1) / kTile : 0;
 }
 
@@ -65,12 +65,14 @@ extern "C" mla_status_t mla_get_metadata_host(const int32_t* cache_seqlens, int 
   if (topk < 0 || (topk > 0 && topk % 64 != 0)) return MLA_ERR_INVALID_ARG;
   if (topk == 0 && !cache_seqlens) return MLA_ERR_INVALID_ARG;
   if (h_kv != 1) return MLA_ERR_UNSUPPORTED;
-  const int U = topk > 0 ? batch * s_q : batch;
+  Geometry g;
+  if (!unit_geometry(s_q, h_q, h_kv, topk, &g)) return MLA_ERR_UNSUPPORTED;
+  const int U = batch * g.units_per_req;
   // cost prefix C[0..U] kept in num_splits first, then replaced by split pointers
   int total = 0, max_cost = 0;
   for (int u = 0; u < U; ++u) {
     num_splits[u] = (int32_t)total;
-    int n = unit_tiles(cache_seqlens, u, topk);
+    int n = unit_tiles(cache_seqlens, u, g.units_per_req, topk);
     const int cost = n > 0 ? n + kSchedOverhead : 0;
     total += cost;
     max_cost = cost > max_cost ? cost : max_cost;
@@ -88,7 +90,7 @@ extern "C" mla_status_t mla_get_metadata_host(const int32_t* cache_seqlens, int 
   int32_t acc = 0;
   for (int u = 0; u < U; ++u) {
     const int Cu = num_splits[u];
-    const int n = unit_tiles(cache_seqlens, u, topk);
+    const int n = unit_tiles(cache_seqlens, u, g.units_per_req, topk);
     int ns = 0;
     if (n > 0) ns = (int)((Cu + kSchedOverhead + n - 1) / payload) - first_part_of(Cu, payload) + 1;
     num_splits[u] = acc;
@@ -148,7 +150,7 @@ __device__ int block_max(int v) {
 }
 
 __global__ void __launch_bounds__(kMetaThreads) mla_metadata_kernel(const int32_t* __restrict__ seqlens,
-                                                                   int U, int topk, int parts,
+                                                                   int U, int upr, int topk, int parts,
                                                                    int32_t* __restrict__ tile_md,
                                                                    int32_t* __restrict__ num_splits) {
   __shared__ int s_payload;
@@ -158,7 +160,7 @@ __global__ void __launch_bounds__(kMetaThreads) mla_metadata_kernel(const int32_
   // 1. cost prefix C[u] -> num_splits[u], total -> num_splits[U]
   int my = 0, my_max = 0;
   for (int u = u0; u < u1; ++u) {
-    int n = unit_tiles(seqlens, u, topk);
+    int n = unit_tiles(seqlens, u, upr, topk);
     const int cost = n > 0 ? n + kSchedOverhead : 0;
     my += cost;
     my_max = max(my_max, cost);
@@ -169,7 +171,7 @@ __global__ void __launch_bounds__(kMetaThreads) mla_metadata_kernel(const int32_
   int c = sc.x;
   for (int u = u0; u < u1; ++u) {
     num_splits[u] = c;
-    int n = unit_tiles(seqlens, u, topk);
+    int n = unit_tiles(seqlens, u, upr, topk);
     c += n > 0 ? n + kSchedOverhead : 0;
   }
   if (t == 0) {
@@ -192,7 +194,7 @@ __global__ void __launch_bounds__(kMetaThreads) mla_metadata_kernel(const int32_
   int mys = 0;
   for (int u = u0; u < u1; ++u) {
     const int Cu = num_splits[u];
-    const int n = unit_tiles(seqlens, u, topk);
+    const int n = unit_tiles(seqlens, u, upr, topk);
     if (n > 0) mys += (int)((Cu + kSchedOverhead + n - 1) / payload) - first_part_of(Cu, payload) + 1;
   }
   const int2 ss = block_exclusive_scan(mys);
@@ -200,7 +202,7 @@ __global__ void __launch_bounds__(kMetaThreads) mla_metadata_kernel(const int32_
   int sp = ss.x;
   for (int u = u0; u < u1; ++u) {
     const int Cu = num_splits[u];  // read before overwriting this slot
-    const int n = unit_tiles(seqlens, u, topk);
+    const int n = unit_tiles(seqlens, u, upr, topk);
     int ns = 0;
     if (n > 0) ns = (int)((Cu + kSchedOverhead + n - 1) / payload) - first_part_of(Cu, payload) + 1;
     num_splits[u] = sp;
@@ -216,9 +218,9 @@ __global__ void __launch_bounds__(kMetaThreads) mla_metadata_kernel(const int32_
   }
 }
 
-mla_status_t launch_metadata(const int32_t* seqlens, int U, int topk, int parts, int32_t* tile_md,
+mla_status_t launch_metadata(const int32_t* seqlens, int U, int upr, int topk, int parts, int32_t* tile_md,
                              int32_t* num_splits, cudaStream_t stream) {
-  mla_metadata_kernel<<<1, kMetaThreads, 0, stream>>>(seqlens, U, topk, parts, tile_md, num_splits);
+  mla_metadata_kernel<<<1, kMetaThreads, 0, stream>>>(seqlens, U, upr, topk, parts, tile_md, num_splits);
   return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 

@@ -22,8 +22,8 @@ class DecodeRunner:
         assert d == 576
         self.topk = int(indices.shape[-1]) if indices is not None else 0
         self.kv_format = C.MLA_KV_BF16 if kcache.dtype == torch.bfloat16 else C.MLA_KV_FP8_E4M3
-        self.units = self.batch * self.s_q if self.topk else self.batch
-        self.rows = self.h_q if self.topk else self.s_q * self.h_q
+        upr, self.rows = C.mla_decode_geometry(self.s_q, self.h_q, 1, self.topk)
+        self.units = self.batch * upr
         self.parts = num_sm_parts or C.mla_get_num_sm_parts(dev.index or 0, self.s_q, self.h_q, 1, self.topk)
         self.tile_md = torch.empty(self.parts * C.MLA_TILE_MD_INTS, dtype=torch.int32, device=dev)
         self.num_splits = torch.empty(self.units + 1, dtype=torch.int32, device=dev)

@@ -101,23 +101,39 @@ enum {
 #define MLA_D_V 512
 #define MLA_PAGE_SIZE 64
 #define MLA_TILE_MD_INTS 8 /* int32 entries per scheduler part */
-#define MLA_MAX_ROWS 128   /* max query rows (s_q*h_q/h_kv, or h_q when sparse) */
+#define MLA_MAX_ROWS 128   /* max query rows of one work unit */
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char* mla_status_string(mla_status_t status);
 
+/* Work units of a decode problem (host-only, pure function of the sizes).
+ * Paged decoding (topk == 0): the R = s_q*h_q/h_kv query rows of a request,
+ * laid out [query token][head], are cut into the fewest equal blocks of at
+ * most MLA_MAX_ROWS rows (the smallest count n >= ceil(R/128) that divides
+ * R); every block is a unit of R/n rows that reads the request's whole key
+ * set (FlashInfer README: q_len query tokens per request, six for
+ * DeepSeek-V4, so R reaches 6*64 = 384 rows). Sparse decoding (topk > 0):
+ * one unit per (request, query token) of h_q/h_kv rows. The units of a
+ * request are consecutive: unit u is rows [u*rows, (u+1)*rows) of the
+ * flattened [batch*s_q*h_q] row axis of q, out and lse.
+ * Writes *units_per_request (units = batch * units_per_request) and
+ * *rows_per_unit. Errors: INVALID_ARG (null outputs, non-positive sizes),
+ * UNSUPPORTED (h_kv != 1; sparse h_q > MLA_MAX_ROWS; s_q*h_q > 2^20). */
+mla_status_t mla_decode_geometry(int s_q, int h_q, int h_kv, int topk, int* units_per_request,
+                                 int* rows_per_unit);
+
 /* Number of scheduler parts for a problem on `device` (host-only query).
- * rows = s_q*h_q/h_kv for paged decoding, h_q for sparse decoding
- * (topk > 0). One part is processed by ceil(rows/64) CTAs, one per SM, so
- * parts = floor(num_SMs / ceil(rows/64)). Writes *num_sm_parts. */
+ * rows = the rows per unit of mla_decode_geometry. One part is processed by
+ * ceil(rows/64) CTAs, one per SM, so parts = floor(num_SMs / ceil(rows/64))
+ * (for two CTAs per part, no more than the CTA pairs that fit at once).
+ * Writes *num_sm_parts. */
 mla_status_t mla_get_num_sm_parts(int device, int s_q, int h_q, int h_kv, int topk, int* num_sm_parts);
 
 /* Split-KV tile scheduler ("get_mla_metadata" in the pages' API).
  *
- * Work units: paged decoding (topk == 0) has one unit per request b with
- * ceil(cache_seqlens[b]/128) blocks of 128 tokens (two pages); sparse
- * decoding (topk > 0) has one unit per (b, i), i < s_q, with ceil(topk/128)
- * blocks of 128 index slots. Every unit costs its blocks plus a fixed
+ * Work units (mla_decode_geometry): a paged unit of request b has
+ * ceil(cache_seqlens[b]/128) blocks of 128 tokens (two pages); a sparse
+ * unit (b, i), i < s_q, has ceil(topk/128) blocks of 128 index slots. Every unit costs its blocks plus a fixed
  * overhead of 3 blocks; the units are laid end to end and cut into ranges of
  * equal cost, so one part covers a contiguous run of (unit, block) pairs and
  * a unit may be split across parts. The range length is
@@ -136,7 +152,7 @@ mla_status_t mla_get_num_sm_parts(int device, int s_q, int h_q, int h_kv, int to
  *                  no blocks has 0 splits).
  * Both outputs are reusable by every layer of the same decode step.
  * Errors: INVALID_ARG for null outputs or non-positive sizes, topk % 64 != 0;
- * UNSUPPORTED for h_kv != 1. */
+ * UNSUPPORTED for h_kv != 1 or s_q*h_q > 2^20. */
 mla_status_t mla_get_metadata(const int32_t* cache_seqlens, int batch, int s_q, int h_q, int h_kv,
                               int topk, int num_sm_parts, int32_t* tile_md, int32_t* num_splits,
                               mla_stream_t stream);
@@ -146,7 +162,8 @@ mla_status_t mla_get_metadata(const int32_t* cache_seqlens, int batch, int s_q, 
 mla_status_t mla_get_metadata_host(const int32_t* cache_seqlens, int batch, int s_q, int h_q, int h_kv,
                                    int topk, int num_sm_parts, int32_t* tile_md, int32_t* num_splits);
 
-/* Bytes of caller-owned workspace a decode call needs:
+/* Bytes of caller-owned workspace a decode call needs (units and rows as
+ * given by mla_decode_geometry):
  *   256-byte header (the device status word at offset 0), then
  *   partial LSE  fp32 [units + num_sm_parts][rows]          (256-B aligned)
  *   partial O    fp32 [units + num_sm_parts][rows][512]     (256-B aligned)
@@ -195,8 +212,8 @@ typedef struct {
  * Output rows of units processed in one piece are written by the decode
  * kernel; split units and empty units are finished by the combine. Errors:
  * INVALID_ARG (null or misaligned pointers, d_qk/d_v/page_size mismatch,
- * non-positive sizes, bad kv_format), UNSUPPORTED (h_kv != 1, rows >
- * MLA_MAX_ROWS), WORKSPACE_TOO_SMALL, CUDA (launch failure). */
+ * non-positive sizes, bad kv_format), UNSUPPORTED (h_kv != 1, s_q*h_q >
+ * 2^20), WORKSPACE_TOO_SMALL, CUDA (launch failure). */
 mla_status_t mla_decode_paged(const mla_decode_args* args, mla_stream_t stream);
 
 /* Paged decoding with a built-in workspace (the pages have no counterpart:
@@ -230,7 +247,8 @@ mla_status_t mla_decode_paged_noalloc(const mla_decode_args* args, mla_stream_t 
  * and set MLA_DEVICE_STATUS_BOUNDS; duplicates count as often as they occur.
  * topk must be a positive multiple of 64; `causal` is ignored; kv_format must
  * be MLA_KV_BF16. tile_md/num_splits come from mla_get_metadata(..., topk).
- * Errors as for mla_decode_paged. */
+ * Errors as for mla_decode_paged; UNSUPPORTED also for h_q/h_kv >
+ * MLA_MAX_ROWS. */
 mla_status_t mla_decode_sparse(const mla_decode_args* args, const int32_t* indices, int topk,
                                mla_stream_t stream);
 
@@ -239,21 +257,21 @@ mla_status_t mla_decode_sparse(const mla_decode_args* args, const int32_t* indic
  *   n >= 2: lse = ln sum_s exp(lse_s), out = sum_s exp(lse_s - lse) * o_s
  *           over the workspace partials (fp32), out rounded to bf16;
  *   n == 0: out = 0, lse = -inf;   n == 1: nothing is written.
- * out/lse rows of unit u start at row u*rows_per_unit (rows = s_q*h_q for
- * paged units, h_q for sparse units; see mla_workspace_size). */
+ * out/lse rows of unit u start at row u*rows_per_unit (units and rows as
+ * given by mla_decode_geometry). */
 mla_status_t mla_combine(const void* workspace, size_t workspace_bytes, const int32_t* num_splits,
                          int num_units, int rows_per_unit, int num_sm_parts, void* out, float* lse,
                          mla_stream_t stream);
 
 /* mla_combine with a per-head attention sink (see mla_decode_args.sink):
- * after the splits are merged, row r of a unit (head r % h_q) takes
- *   lse' = ln(e^lse + e^sink[r % h_q]),  out *= e^(lse - lse'),
- * and a unit with n == 0 gets out = 0, lse = sink[r % h_q]. Units with
- * n == 1 are left alone (their decode piece folded the sink in already).
+ * after the splits are merged, row r of unit u, whose head is
+ * h = (u*rows_per_unit + r) % h_q, takes
+ *   lse' = ln(e^lse + e^sink[h]),  out *= e^(lse - lse'),
+ * and a unit with n == 0 gets out = 0, lse = sink[h]. Units with n == 1 are
+ * left alone (their decode piece folded the sink in already).
  * sink: device fp32 [h_q], 4-B aligned, or NULL (then identical to
  * mla_combine and h_q is ignored). Errors as mla_combine; INVALID_ARG also
- * when sink is given and h_q <= 0, rows_per_unit % h_q != 0 or sink is
- * misaligned. */
+ * when sink is given and h_q <= 0 or sink is misaligned. */
 mla_status_t mla_combine_sink(const void* workspace, size_t workspace_bytes, const int32_t* num_splits,
                               int num_units, int rows_per_unit, int num_sm_parts, int h_q, const float* sink,
                               void* out, float* lse, mla_stream_t stream);

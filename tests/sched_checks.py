@@ -13,10 +13,26 @@ OVERHEAD = 3
 SPLIT_PENALTY = 8
 
 
-def unit_tiles(seqlens, batch, s_q, topk):
+MAX_ROWS = 128
+
+
+def units_per_request(s_q, h_q, topk):
+    """Paged: the fewest equal blocks of <= 128 rows that cut s_q*h_q rows;
+    sparse: one unit per query token."""
+    if topk or h_q is None:
+        return s_q if topk else 1
+    R = s_q * h_q
+    n = -(-R // MAX_ROWS)
+    while R % n:
+        n += 1
+    return n
+
+
+def unit_tiles(seqlens, batch, s_q, topk, h_q=None):
     if topk:
         return [(topk + TILE - 1) // TILE] * (batch * s_q)
-    return [max(0, (int(L) + TILE - 1) // TILE) for L in seqlens[:batch]]
+    upr = units_per_request(s_q, h_q, topk)
+    return [max(0, (int(seqlens[u // upr]) + TILE - 1) // TILE) for u in range(batch * upr)]
 
 
 def pieces_of_part(md, n):
@@ -33,8 +49,9 @@ def pieces_of_part(md, n):
     return out
 
 
-def check_schedule(tile_md, num_splits, seqlens, batch, s_q, topk, parts):
-    n = unit_tiles(seqlens, batch, s_q, topk)
+def check_schedule(tile_md, num_splits, seqlens, batch, s_q, topk, parts, h_q=None):
+    """h_q=None: one unit per request (s_q*h_q <= 128) on the paged path."""
+    n = unit_tiles(seqlens, batch, s_q, topk, h_q)
     U = len(n)
     md = np.asarray(tile_md).reshape(parts, 8)
     ptr = np.asarray(num_splits)[:U + 1]

@@ -76,8 +76,7 @@ def _fake_args(**over):
     (dict(kv_format=7), C.MLA_ERR_INVALID_ARG),
     (dict(softmax_scale=float("nan")), C.MLA_ERR_INVALID_ARG),
     (dict(h_kv=2, h_q=32), C.MLA_ERR_UNSUPPORTED),
-    (dict(h_q=256), C.MLA_ERR_UNSUPPORTED),
-    (dict(s_q=2, h_q=128), C.MLA_ERR_UNSUPPORTED),
+    (dict(s_q=1 << 11, h_q=1 << 10), C.MLA_ERR_UNSUPPORTED),  # more than 2^20 rows per request
     (dict(workspace_bytes=1024), C.MLA_ERR_WORKSPACE_TOO_SMALL),
     (dict(sink=0x300002), C.MLA_ERR_INVALID_ARG),             # misaligned sink
 ])
@@ -94,6 +93,8 @@ def test_sparse_rejects_bad_topk_and_fp8():
     a8 = _fake_args(kv_format=C.MLA_KV_FP8_E4M3)
     assert L.mla_decode_sparse(ctypes.byref(a8), 0x200000, 128, None) == C.MLA_ERR_UNSUPPORTED
     assert L.mla_decode_paged(None, None) == C.MLA_ERR_INVALID_ARG
+    a256 = _fake_args(h_q=256)                        # sparse units are one query token: <= 128 rows
+    assert L.mla_decode_sparse(ctypes.byref(a256), 0x200000, 128, None) == C.MLA_ERR_UNSUPPORTED
 
 
 def test_metadata_rejects_bad_arguments():
@@ -105,14 +106,38 @@ def test_metadata_rejects_bad_arguments():
     assert L.mla_combine(None, 0, None, 1, 1, 1, None, None, None) == C.MLA_ERR_INVALID_ARG
     ws, ns, out, lse, sink = 0x100000, 0x200000, 0x300000, 0x400000, 0x500000
     big = 1 << 40
-    for h_q, sk in ((0, sink), (3, sink), (16, sink + 2)):   # h_q <= 0, rows % h_q, misaligned
+    for h_q, sk in ((0, sink), (16, sink + 2)):   # h_q <= 0, misaligned
         assert L.mla_combine_sink(ws, big, ns, 4, 32, 8, h_q, sk, out, lse, None) == C.MLA_ERR_INVALID_ARG
     assert L.mla_combine_sink(ws, 1024, ns, 4, 32, 8, 16, sink, out, lse, None) == C.MLA_ERR_WORKSPACE_TOO_SMALL
     assert L.mla_query_device_status(None, None, None) == C.MLA_ERR_INVALID_ARG
 
 
+@pytest.mark.parametrize("s_q,h_q,topk,expect", [
+    (1, 128, 0, (1, 128)), (2, 16, 0, (1, 32)), (6, 16, 0, (1, 96)), (6, 64, 0, (3, 128)),
+    (3, 64, 0, (2, 96)), (1, 256, 0, (2, 128)), (3, 43, 0, (3, 43)), (5, 32, 0, (2, 80)),
+    (4, 128, 0, (4, 128)), (2, 128, 2048, (2, 128)), (3, 64, 128, (3, 64)),
+])
+def test_decode_geometry(s_q, h_q, topk, expect):
+    assert M.mla_decode_geometry(s_q, h_q, 1, topk) == expect
+    assert S.units_per_request(s_q, h_q, topk) == expect[0]
+    U, R = expect[0], expect[1]
+    lse = (U + 8) * R * 4
+    o_off = -(-(256 + lse) // 256) * 256
+    assert M.mla_workspace_size(1, s_q, h_q, 1, topk, 8) == -(-(o_off + (U + 8) * R * 512 * 4) // 256) * 256
+
+
+def test_decode_geometry_rejects():
+    L = C.lib()
+    a, b = ctypes.c_int(0), ctypes.c_int(0)
+    assert L.mla_decode_geometry(1, 256, 1, 128, ctypes.byref(a), ctypes.byref(b)) == C.MLA_ERR_UNSUPPORTED
+    assert L.mla_decode_geometry(1 << 11, 1 << 10, 1, 0, ctypes.byref(a), ctypes.byref(b)) == C.MLA_ERR_UNSUPPORTED
+    assert L.mla_decode_geometry(1, 16, 2, 0, ctypes.byref(a), ctypes.byref(b)) == C.MLA_ERR_UNSUPPORTED
+    assert L.mla_decode_geometry(0, 16, 1, 0, ctypes.byref(a), ctypes.byref(b)) == C.MLA_ERR_INVALID_ARG
+    assert L.mla_decode_geometry(1, 16, 1, 0, None, ctypes.byref(b)) == C.MLA_ERR_INVALID_ARG
+
+
 def host_schedule(seqlens, batch, s_q, h_q, topk, parts):
-    U = batch * s_q if topk else batch
+    U = batch * M.mla_decode_geometry(s_q, h_q, 1, topk)[0]
     md = np.zeros(parts * 8, dtype=np.int32)
     ns = np.zeros(U + 1, dtype=np.int32)
     sl = np.ascontiguousarray(np.asarray(seqlens, dtype=np.int32))
@@ -129,11 +154,14 @@ def host_schedule(seqlens, batch, s_q, h_q, topk, parts):
     ("more_parts_than_tiles", [1, 2, 3], 1, 64, 0, 148),
     ("sparse", [32768] * 32, 1, 128, 2048, 74),
     ("sparse_sq2", [4096] * 3, 2, 64, 192, 11),
+    ("mtp6_64heads", [4096, 300, 0, 9000], 6, 64, 0, 74),
+    ("rows96_blocks", [70, 129, 5000], 3, 64, 0, 74),
+    ("256heads", [4096] * 8, 1, 256, 0, 74),
 ])
 def test_host_scheduler_invariants(case):
     _, lens, s_q, h_q, topk, parts = case
     md, ns = host_schedule(lens, len(lens), s_q, h_q, topk, parts)
-    S.check_schedule(md, ns, lens, len(lens), s_q, topk, parts)
+    S.check_schedule(md, ns, lens, len(lens), s_q, topk, parts, h_q=h_q)
 
 
 def test_host_scheduler_random_and_mtp():

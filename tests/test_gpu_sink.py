@@ -29,7 +29,7 @@ def _sparse(batch, seqlens, s_q, h_q, topk, neg_frac=0.05, seed=1):
 def _check(inp, where, **kw):
     out, lse, r = G.run_gpu(inp, runner_kwargs=kw)
     ref_o, ref_l = G.oracle_for(inp)
-    info = G.compare(out, lse, ref_o, ref_l, where)
+    info = G.compare(out, lse, ref_o, ref_l, where, inp=inp)
     assert r.status()[0] == C.MLA_OK
     return out, lse, info
 
