@@ -84,7 +84,8 @@ mla_status_t run_decode(const mla_decode_args* a, const int32_t* indices, int to
   const Geometry g = geometry_of(a->s_q, a->h_q, a->h_kv, topk);
   const int rows = g.rows;
   const int U = a->batch * g.units_per_req;
-  const int mode = topk > 0 ? kModeSparse : (a->kv_format == MLA_KV_FP8_E4M3 ? kModeFp8 : kModeBf16);
+  const bool fp8 = a->kv_format == MLA_KV_FP8_E4M3;
+  const int mode = topk > 0 ? (fp8 ? kModeFp8Sparse : kModeSparse) : (fp8 ? kModeFp8 : kModeBf16);
   // Q rows of every unit, and (bf16 paged cache only) the cache as
   // [pages*64 tokens][576 dims]; boxes of 64 x 64 with 128-B swizzle. The FP8
   // and sparse modes read the cache with cp.async and need no cache map.
@@ -94,7 +95,7 @@ mla_status_t run_decode(const mla_decode_args* a, const int32_t* indices, int to
   const int row_groups = (rows + kRowsPerCta - 1) / kRowsPerCta;
   // more than 64 rows on the BF16 cache (paged or sparse): one CTA pair per
   // part shares each cache tile between the two row halves
-  const bool pair = row_groups == 2 && mode != kModeFp8;
+  const bool pair = row_groups == 2 && !mode_fp8(mode);
   if (mode == kModeBf16 &&
       !make_map(&tkv, a->kcache, (uint64_t)a->num_pages * kPage, kDqk, kDqk * 2, 64, 64))
     return MLA_ERR_CUDA;
@@ -219,7 +220,6 @@ mla_status_t mla_decode_sparse(const mla_decode_args* args, const int32_t* indic
   if (!indices || topk <= 0 || topk % 64 != 0) return MLA_ERR_INVALID_ARG;
   mla_status_t st = check_common(args, topk);
   if (st != MLA_OK) return st;
-  if (args->kv_format != MLA_KV_BF16) return MLA_ERR_UNSUPPORTED;
   return run_decode(args, indices, topk, reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -126,7 +126,7 @@ template <int MODE, bool KGROUP>
 __device__ __forceinline__ void retire_slot(const GatherRing& g, int seq, int lw, int t) {
   const int slot = seq % g.nslots;
   uint8_t* s = g.base + slot * kSlot;
-  if (MODE == kModeFp8) {
+  if (mode_fp8(MODE)) {
     __syncwarp();  // every lane's copies of this slot are complete and visible
     if (KGROUP) {
       const int j = seq % 9;
@@ -169,14 +169,16 @@ __device__ __forceinline__ void retire_slot(const GatherRing& g, int seq, int lw
 }
 
 // Source row of tile-relative token tt of tile k (FP8 record, or bf16 cache
-// row for sparse; ok = 0 for an ignored sparse slot, which is zero-filled).
+// row; ok = 0 for an ignored sparse slot, whose copies zero-fill: codes and
+// scales 0 dequantise to 0 as well).
 template <int MODE, bool KGROUP>
 __device__ __forceinline__ const uint8_t* gather_src(const DecodeParams& p, int unit, int req, int npg, int k, int tt,
                                                      uint32_t& ok) {
-  if (MODE == kModeSparse) {
+  if (mode_sparse(MODE)) {
     const int row = sparse_row(p, unit, k * kTile + tt, KGROUP);
     ok = row >= 0 ? 16u : 0u;
-    return static_cast<const uint8_t*>(p.kcache) + (size_t)(row >= 0 ? row : 0) * (kDqk * 2);
+    const size_t rb = MODE == kModeSparse ? (size_t)kDqk * 2 : (size_t)kFp8RecordBytes;
+    return static_cast<const uint8_t*>(p.kcache) + (size_t)(row >= 0 ? row : 0) * rb;
   }
   int pg = page_of(p, req, 2 * k + (tt >> 6), npg);
   if (pg < 0) pg = page_of(p, req, 2 * k, npg);  // half tile: page A again (keys masked, values zero-filled later)
@@ -193,7 +195,7 @@ __device__ void gather_group(const DecodeParams& p, Ctrl* c, PieceIter& it, cons
   while (!stop && it.next(pc)) {
     const int unit = pc.unit;
     const int req = unit_req(p, unit);
-    const int npg = (MODE == kModeSparse) ? 0 : (p.seqlens[req] + kPage - 1) / kPage;
+    const int npg = mode_sparse(MODE) ? 0 : (p.seqlens[req] + kPage - 1) / kPage;
     for (int k = pc.t0; k < pc.t1 && !stop; ++k) {
       // K: lane t owns tile row 32lw + t; V: lane t (< 16) owns row 16lw + t
       // of page h, i.e. tile row 64h + 16lw + t
@@ -225,9 +227,10 @@ __device__ void gather_group(const DecodeParams& p, Ctrl* c, PieceIter& it, cons
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const int r = 8 * i + (t >> 2), cc = t & 3;
-              cp_async16(s + (32 * lw + r) * 128 + 16 * cc, shfl_ptr(srcK, r) + 64 * j + 16 * cc, 16u);
+              const uint32_t nb = __shfl_sync(0xffffffffu, ok, r);
+              cp_async16(s + (32 * lw + r) * 128 + 16 * cc, shfl_ptr(srcK, r) + 64 * j + 16 * cc, nb);
             }
-            cp_async16(s + (32 * lw + t) * 128 + 64, srcK + 512, 16u);
+            cp_async16(s + (32 * lw + t) * 128 + 64, srcK + 512, ok);
           }
         } else {  // V slot j: value dims 128*(j/2).., page half h = j%2
           const int m = j >> 1;
@@ -244,9 +247,10 @@ __device__ void gather_group(const DecodeParams& p, Ctrl* c, PieceIter& it, cons
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const int r = 4 * i + (t >> 3), ch = t & 7;
-              cp_async16(s + (16 * lw + r) * 128 + 16 * ch, shfl_ptr(sv, r) + 128 * m + 16 * ch, 16u);
+              const uint32_t nb = __shfl_sync(0xffffffffu, okv, r);
+              cp_async16(s + (16 * lw + r) * 128 + 16 * ch, shfl_ptr(sv, r) + 128 * m + 16 * ch, nb);
             }
-            if (t < 16) cp_async16(s + 8192 + (16 * lw + t) * 128, sv + 512, 16u);
+            if (t < 16) cp_async16(s + 8192 + (16 * lw + t) * 128, sv + 512, okv);
           }
         }
         cp_async_commit();
@@ -449,7 +453,7 @@ __global__ void __launch_bounds__(MODE == kModeBf16 ? 256 : 256 + 2 * kGatherThr
         if (stop) break;
         // dense: value rows of keys past the request's end must read as zero
         // (ignored sparse slots are zero-filled by the gather already)
-        const int nvalid = (MODE == kModeSparse) ? kTile : dense_tile_valid(p.seqlens[req], k);
+        const int nvalid = mode_sparse(MODE) ? kTile : dense_tile_valid(p.seqlens[req], k);
         const uint32_t pt = smem_u32(sP);
         for (int j = 0; j < 8 && !stop; ++j, ++vc) {
           const int slot = vc % kNV;
@@ -504,7 +508,7 @@ __global__ void __launch_bounds__(MODE == kModeBf16 ? 256 : 256 + 2 * kGatherThr
       const int req = unit_req(p, pc.unit);
       const int grow = row0 + r;                          // row within the unit
       int limit = 0;
-      if (MODE != kModeSparse) {
+      if (!mode_sparse(MODE)) {
         const int Ls = p.seqlens[req];
         limit = Ls;
         if (p.causal) limit = Ls - p.s_q + row_query(p, pc.unit, grow) + 1;
@@ -515,7 +519,7 @@ __global__ void __launch_bounds__(MODE == kModeBf16 ? 256 : 256 + 2 * kGatherThr
         const int b = gt & 1;
         // validity of the 128 keys of this tile for this row (bit i of word w = key 32w + i)
         uint4 vmask;
-        if (MODE == kModeSparse) {
+        if (mode_sparse(MODE)) {
           vmask.x = __ballot_sync(0xffffffffu, sparse_row(p, pc.unit, k * kTile + lane, false) >= 0);
           vmask.y = __ballot_sync(0xffffffffu, sparse_row(p, pc.unit, k * kTile + 32 + lane, false) >= 0);
           vmask.z = __ballot_sync(0xffffffffu, sparse_row(p, pc.unit, k * kTile + 64 + lane, false) >= 0);
@@ -698,7 +702,8 @@ cudaError_t launch_decode(int rows_per_cta, int mode, const CUtensorMap& tq, con
 #define MLA_DISPATCH(NRV)                                                                         \
   if (mode == kModeBf16) return launch_one<NRV, kModeBf16>(tq, tkv, p, parts, row_groups, stream); \
   if (mode == kModeFp8) return launch_one<NRV, kModeFp8>(tq, tkv, p, parts, row_groups, stream);   \
-  return launch_one<NRV, kModeSparse>(tq, tkv, p, parts, row_groups, stream);
+  if (mode == kModeSparse) return launch_one<NRV, kModeSparse>(tq, tkv, p, parts, row_groups, stream); \
+  return launch_one<NRV, kModeFp8Sparse>(tq, tkv, p, parts, row_groups, stream);
   // <= 16 rows run in the 32-row kernel: the extra P^T rows are written as
   // zeros and their output rows are never stored
   if (rows_per_cta <= 32) { MLA_DISPATCH(32) }

@@ -7,7 +7,11 @@
 
 namespace mla {
 
-enum KvMode : int { kModeBf16 = 0, kModeFp8 = 1, kModeSparse = 2 };
+// Cache format x key-set kind: BF16 paged, FP8 paged, BF16 token-sparse,
+// FP8 token-sparse.
+enum KvMode : int { kModeBf16 = 0, kModeFp8 = 1, kModeSparse = 2, kModeFp8Sparse = 3 };
+__host__ __device__ constexpr bool mode_fp8(int mode) { return mode == kModeFp8 || mode == kModeFp8Sparse; }
+__host__ __device__ constexpr bool mode_sparse(int mode) { return mode == kModeSparse || mode == kModeFp8Sparse; }
 
 struct DecodeParams {
   int units, rows, h_q, s_q, causal, topk;  // rows = query rows per unit

@@ -245,8 +245,11 @@ mla_status_t mla_decode_paged_noalloc(const mla_decode_args* args, mla_stream_t 
  * token positions of request b resolved through its block-table row; -1
  * entries are ignored; other values outside [0, cache_seqlens[b]) are ignored
  * and set MLA_DEVICE_STATUS_BOUNDS; duplicates count as often as they occur.
- * topk must be a positive multiple of 64; `causal` is ignored; kv_format must
- * be MLA_KV_BF16. tile_md/num_splits come from mla_get_metadata(..., topk).
+ * topk must be a positive multiple of 64; `causal` is ignored. Both cache
+ * formats are accepted: with MLA_KV_FP8_E4M3 the indexed token records are
+ * gathered and dequantised as for paged decoding (the FP8 token-sparse
+ * combination of the pages' sparse-decoding figures). tile_md/num_splits
+ * come from mla_get_metadata(..., topk).
  * Errors as for mla_decode_paged; UNSUPPORTED also for h_q/h_kv >
  * MLA_MAX_ROWS. */
 mla_status_t mla_decode_sparse(const mla_decode_args* args, const int32_t* indices, int topk,

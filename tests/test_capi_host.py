@@ -85,13 +85,11 @@ def test_decode_rejects_bad_arguments(over, code):
     assert C.lib().mla_decode_paged(ctypes.byref(a), None) == code
 
 
-def test_sparse_rejects_bad_topk_and_fp8():
+def test_sparse_rejects_bad_topk_and_rows():
     a = _fake_args()
     L = C.lib()
     assert L.mla_decode_sparse(ctypes.byref(a), 0x200000, 100, None) == C.MLA_ERR_INVALID_ARG
     assert L.mla_decode_sparse(ctypes.byref(a), None, 128, None) == C.MLA_ERR_INVALID_ARG
-    a8 = _fake_args(kv_format=C.MLA_KV_FP8_E4M3)
-    assert L.mla_decode_sparse(ctypes.byref(a8), 0x200000, 128, None) == C.MLA_ERR_UNSUPPORTED
     assert L.mla_decode_paged(None, None) == C.MLA_ERR_INVALID_ARG
     a256 = _fake_args(h_q=256)                        # sparse units are one query token: <= 128 rows
     assert L.mla_decode_sparse(ctypes.byref(a256), 0x200000, 128, None) == C.MLA_ERR_UNSUPPORTED
