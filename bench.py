@@ -60,8 +60,9 @@ def kernel_source_hash() -> str:
 
 def decode_kernel_name(w, rows: int) -> str:
     """The decode kernel the library launches for this workload: CTA pairs for
-    units of 65-128 rows on the BF16 paged cache, one CTA per row group otherwise."""
-    if w.kv == "bf16" and not w.topk and rows > 64:
+    units of 65-128 rows on the BF16 cache (paged or token-sparse), one CTA per
+    row group otherwise."""
+    if w.kv == "bf16" and rows > 64:
         return "mla_decode_pair_kernel"
     return "mla_decode_kernel"
 
@@ -144,6 +145,8 @@ def workload_config(inp, work):
                inp.kcache.numel() * inp.kcache.element_size() / 1e6)}
     if w.topk:
         cfg["topk"] = w.topk
+    if inp.sink is not None:
+        cfg["sink"] = "seeded per-head logits, N(0,1) + 1"
     return cfg
 
 
@@ -225,6 +228,8 @@ def run_gpu(args):
         pg = dist
 
     inp = W.make_inputs(W.get_workload(args.workload))
+    if args.sink:
+        inp = W.with_sink(inp, seed=inp.workload.seed)
     work = W.algorithmic_work(inp)
     w = inp.workload
     q = inp.q.to(dev)
@@ -232,7 +237,8 @@ def run_gpu(args):
     bt = inp.block_table.to(dev)
     sl = inp.cache_seqlens.to(dev)
     idx = inp.indices.to(dev) if inp.indices is not None else None
-    runner = M.DecodeRunner(q, kc, bt, sl, softmax_scale=w.scale, causal=w.causal, indices=idx)
+    sink = inp.sink.to(dev) if inp.sink is not None else None
+    runner = M.DecodeRunner(q, kc, bt, sl, softmax_scale=w.scale, causal=w.causal, indices=idx, sink=sink)
     # timing variant: the decode kernel alone, then the combine enqueued by the caller
     runner.args.debug_flags = C.MLA_DEBUG_SKIP_COMBINE
     U, R, P = runner.units, runner.rows, runner.parts
@@ -248,7 +254,8 @@ def run_gpu(args):
         runner.run(stream)
         if ev is not None:
             ev[2].record(stream)
-        M.mla_combine(runner.workspace, ws_bytes, runner.num_splits, U, R, P, runner.out, runner.lse, stream)
+        M.mla_combine_sink(runner.workspace, ws_bytes, runner.num_splits, U, R, P, w.h_q, sink, runner.out,
+                           runner.lse, stream)
         if ev is not None:
             ev[3].record(stream)
 
@@ -297,7 +304,7 @@ def run_gpu(args):
     idx_h = inp.indices.pin_memory() if inp.indices is not None else None
     out_h = torch.empty(runner.out.shape, dtype=runner.out.dtype).pin_memory()
     lse_h = torch.empty(runner.lse.shape, dtype=runner.lse.dtype).pin_memory()
-    runner_e2e = M.DecodeRunner(q, kc, bt, sl, softmax_scale=w.scale, causal=w.causal, indices=idx)
+    runner_e2e = M.DecodeRunner(q, kc, bt, sl, softmax_scale=w.scale, causal=w.causal, indices=idx, sink=sink)
 
     def e2e_step():
         q.copy_(q_h, non_blocking=True)
@@ -381,7 +388,9 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="dsv3", choices=[w.name for w in W.named_workloads()])
+    ap.add_argument("--workload", default="dsv3",
+                    choices=[w.name for w in W.named_workloads() + W.extra_workloads()])
+    ap.add_argument("--sink", action="store_true", help="seeded per-head attention-sink logits")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")

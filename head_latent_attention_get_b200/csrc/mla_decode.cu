@@ -220,14 +220,14 @@ __device__ void gather_group(const DecodeParams& p, Ctrl* c, PieceIter& it, cons
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
               const int r = 4 * i + (t >> 3), ch = t & 7;
-              const uint32_t nb = __shfl_sync(0xffffffffu, ok, r);
+              const uint32_t nb = mode_sparse(MODE) ? __shfl_sync(0xffffffffu, ok, r) : 16u;
               cp_async16(sw128(s, 32 * lw + r, ch), shfl_ptr(srcK, r) + off + 16 * ch, nb);
             }
           } else {  // FP8 latent slice j: codes (64 B, 4 lanes per row) and scales, converted at retire
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const int r = 8 * i + (t >> 2), cc = t & 3;
-              const uint32_t nb = __shfl_sync(0xffffffffu, ok, r);
+              const uint32_t nb = mode_sparse(MODE) ? __shfl_sync(0xffffffffu, ok, r) : 16u;
               cp_async16(s + (32 * lw + r) * 128 + 16 * cc, shfl_ptr(srcK, r) + 64 * j + 16 * cc, nb);
             }
             cp_async16(s + (32 * lw + t) * 128 + 64, srcK + 512, ok);
@@ -247,7 +247,7 @@ __device__ void gather_group(const DecodeParams& p, Ctrl* c, PieceIter& it, cons
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const int r = 4 * i + (t >> 3), ch = t & 7;
-              const uint32_t nb = __shfl_sync(0xffffffffu, okv, r);
+              const uint32_t nb = mode_sparse(MODE) ? __shfl_sync(0xffffffffu, okv, r) : 16u;
               cp_async16(s + (16 * lw + r) * 128 + 16 * ch, shfl_ptr(sv, r) + 128 * m + 16 * ch, nb);
             }
             if (t < 16) cp_async16(s + 8192 + (16 * lw + t) * 128, sv + 512, okv);

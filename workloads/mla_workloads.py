@@ -86,8 +86,22 @@ def named_workloads():
     ]
 
 
+def extra_workloads():
+    """Workloads of the rows built beyond the five (seeds 20265+): six query
+    tokens per request at 64 heads (the FlashInfer README's DeepSeek-V4 decode
+    geometry, q_len 6, here on the 576-dim BF16 latent rows), and the
+    token-sparse batch over the FP8 token-record cache."""
+    return [
+        Workload("mtp6", 64, 6, 64, [4096] * 64, causal=True, seed=20265,
+                 note="q_len 6 x 64 heads (384 rows per request), causal, BF16, seqlen 4096"),
+        Workload("fp8_sparse", 32, 1, 128, [32768] * 32, causal=False, kv="fp8", topk=2048,
+                 neg_frac=0.05, seed=20266,
+                 note="token-sparse FP8-record decode, 32768-token caches, topk 2048, 5% -1"),
+    ]
+
+
 def get_workload(name: str) -> Workload:
-    for w in named_workloads():
+    for w in named_workloads() + extra_workloads():
         if w.name == name:
             return w
     raise KeyError(name)
