@@ -44,7 +44,7 @@ namespace mla {
 constexpr int kNK = 4;                 // K ring slots: 128 tokens x 64 dims (16 KB)
 constexpr int kNV = 4;                 // V ring slots: 64 tokens x 128 dims (16 KB)
 constexpr int kSlot = 16384;
-constexpr int kLag = 3;                // gather groups retire a slot 3 slots after issuing it
+constexpr int kLag = 2;                // gather groups retire a slot 2 slots after issuing it
 constexpr int kQBytes = 9 * 8192;      // 64 rows x 576 dims
 constexpr int kTmemCols = 512;
 constexpr int kTmemS = 256;            // S buffers at columns 256 and 384
@@ -131,34 +131,48 @@ __device__ __forceinline__ void retire_slot(const GatherRing& g, int seq, int lw
     if (KGROUP) {
       const int j = seq % 9;
       if (j != 8) {  // latent slice: codes in bytes [0,64) and scales in [64,80) of each row
+        // all reads first (independent loads in flight), one warp barrier,
+        // then every write: the rows are converted in place
+        uint4 cw[4];
+        float sc[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int r = 32 * lw + 8 * i + (t >> 2), cc = t & 3;
-          const uint4 cw = *reinterpret_cast<const uint4*>(s + r * 128 + 16 * cc);
-          const float scale = reinterpret_cast<const float*>(s + r * 128 + 64)[j >> 1];
-          __syncwarp();
+          cw[i] = *reinterpret_cast<const uint4*>(s + r * 128 + 16 * cc);
+          sc[i] = reinterpret_cast<const float*>(s + r * 128 + 64)[j >> 1];
+        }
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = 32 * lw + 8 * i + (t >> 2), cc = t & 3;
           uint4 lo, hi;
-          dequant16(cw, scale, lo, hi);
+          dequant16(cw[i], sc[i], lo, hi);
           *reinterpret_cast<uint4*>(sw128(s, r, 2 * cc)) = lo;
           *reinterpret_cast<uint4*>(sw128(s, r, 2 * cc + 1)) = hi;
         }
       }
     } else {  // V slot: codes in the half-0 row, scales at the start of the half-1 row
       const int m = (seq >> 1) & 3;
+      uint4 cw0[2], cw1[2];
+      float sc[2];
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
         const int r = 16 * lw + 8 * i + (t >> 2), c4 = t & 3;  // codes 32*c4 .. 32*c4+31 of row r
-        const uint4 cw0 = *reinterpret_cast<const uint4*>(s + r * 128 + 32 * c4);
-        const uint4 cw1 = *reinterpret_cast<const uint4*>(s + r * 128 + 32 * c4 + 16);
-        const float scale = reinterpret_cast<const float*>(s + 8192 + r * 128)[m];
-        __syncwarp();
+        cw0[i] = *reinterpret_cast<const uint4*>(s + r * 128 + 32 * c4);
+        cw1[i] = *reinterpret_cast<const uint4*>(s + r * 128 + 32 * c4 + 16);
+        sc[i] = reinterpret_cast<const float*>(s + 8192 + r * 128)[m];
+      }
+      __syncwarp();
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int r = 16 * lw + 8 * i + (t >> 2), c4 = t & 3;
         uint8_t* half = s + (c4 >> 1) * 8192;
         const int c0 = 4 * (c4 & 1);
         uint4 lo, hi;
-        dequant16(cw0, scale, lo, hi);
+        dequant16(cw0[i], sc[i], lo, hi);
         *reinterpret_cast<uint4*>(sw128(half, r, c0)) = lo;
         *reinterpret_cast<uint4*>(sw128(half, r, c0 + 1)) = hi;
-        dequant16(cw1, scale, lo, hi);
+        dequant16(cw1[i], sc[i], lo, hi);
         *reinterpret_cast<uint4*>(sw128(half, r, c0 + 2)) = lo;
         *reinterpret_cast<uint4*>(sw128(half, r, c0 + 3)) = hi;
       }
