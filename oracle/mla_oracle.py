@@ -47,6 +47,17 @@ Readings where the pages are silent (listed in the design doc as well):
   * FP8 record = [512 e4m3 | 4 fp32 scales | 64 bf16 RoPE]; the dequantised
     value is bf16_RNE(fp32(e4m3) * scale) with the fp32 product rounded to
     nearest; the oracle then uses those values exactly in fp64.
+  * NVFP4 ("[flashinfer] FlashInfer, NVFP4를 활용한 DeepSeek-V4 디코딩 성능
+    최적화", section 2, the nvfp4_mla_decode README and its tensor table): the
+    query and the cache rows are 512 values each (d_qk = d_v = 512: the whole
+    row is K and V), E2M1 codes packed two per byte (256 bytes per row) with
+    one UE4M3 scale per block of 16 values (32 bytes per row). Readings: byte
+    i holds element 2i in its low nibble and 2i+1 in its high nibble; scale
+    byte j applies to elements [16j, 16j+16); UE4M3 is E4M3 without the sign
+    bit (bit 7 is not part of the format and is ignored); the value is
+    e2m1(code) * ue4m3(scale), used exactly. The pages' kernel rounds P and a
+    requantised V to FP8 on the way; the oracle is the attention of the
+    dequantised values themselves.
 """
 from __future__ import annotations
 
@@ -104,6 +115,36 @@ def e4m3_to_f64(codes) -> np.ndarray:
     val = np.where(e == 0, (m / 8.0) * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e - 7.0))
     val = sign * val
     return np.where((e == 15) & (m == 7), np.nan, val)
+
+
+def e2m1_to_f64(codes) -> np.ndarray:
+    """OCP FP4 E2M1 code (low 4 bits) -> value: sign bit 3, exponent bits 2..1
+    (bias 1), mantissa bit 0; exponent 0 is subnormal (m * 0.5), otherwise
+    2^(e-1) * (1 + m/2). Magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6."""
+    c = np.asarray(codes).astype(np.int64) & 0xF
+    sign = np.where(c & 0x8, -1.0, 1.0)
+    e = (c >> 1) & 0x3
+    m = c & 0x1
+    mag = np.where(e == 0, 0.5 * m, np.exp2(e - 1.0) * (1.0 + 0.5 * m))
+    return sign * mag
+
+
+def ue4m3_to_f64(codes) -> np.ndarray:
+    """UE4M3 scale byte -> value: the E4M3 value of the low 7 bits (no sign)."""
+    return e4m3_to_f64(np.asarray(codes).astype(np.int64) & 0x7F)
+
+
+NVFP4_BLOCK = 16
+
+
+def dequant_nvfp4(packed, scales) -> np.ndarray:
+    """uint8 packed E2M1 [..., n/2] and UE4M3 block scales [..., n/16] -> fp64
+    [..., n]: element 2i is the low nibble of byte i, 2i+1 the high nibble;
+    element d is scaled by scale byte d // 16."""
+    pk = np.asarray(packed, dtype=np.uint8)
+    codes = np.stack([pk & 0xF, pk >> 4], axis=-1).reshape(*pk.shape[:-1], 2 * pk.shape[-1])
+    sc = ue4m3_to_f64(np.asarray(scales, dtype=np.uint8))
+    return e2m1_to_f64(codes) * np.repeat(sc, NVFP4_BLOCK, axis=-1)
 
 
 def dequant_fp8_records(records) -> np.ndarray:
@@ -264,6 +305,9 @@ def combine(o_parts, lse_parts, sink=None):
 
 def inputs_to_f64(inp):
     """(q fp64, cache fp64) from a workloads.DecodeInputs."""
+    if inp.workload.kv == "nvfp4":
+        return (dequant_nvfp4(inp.q.numpy(), inp.q_scale.numpy()),
+                dequant_nvfp4(inp.kcache.numpy(), inp.kv_scale.numpy()))
     return torch_bf16_to_f64(inp.q), cache_to_f64(inp.kcache)
 
 

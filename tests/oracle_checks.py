@@ -438,3 +438,79 @@ def check_sink_reductions(decode_dense, decode_sparse, attend, combine):
         o, l = combine(np.stack([p[0] for p in parts]), np.stack([p[1] for p in parts]), sink=sink)
         _close(o, o_ref, 1e-13)
         _close(l, l_ref, 1e-13)
+
+
+# ---------------------------------------------------------------- NVFP4 (E2M1 + UE4M3 block 16)
+OCP_E2M1 = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]   # OCP MX FP4 E2M1 magnitudes of codes 0..7
+
+
+def check_e2m1(e2m1_to_f64):
+    """All 16 codes against the OCP MX table; bit 3 is the sign."""
+    got = e2m1_to_f64(np.arange(16))
+    want = np.array(OCP_E2M1 + [-x for x in OCP_E2M1])
+    assert np.array_equal(got, want), (got, want)
+    assert np.signbit(got[8]) and not np.signbit(got[0])
+
+
+def check_ue4m3(ue4m3_to_f64):
+    """All 128 scale codes against torch's float8_e4m3fn; bit 7 is ignored."""
+    codes = np.arange(128, dtype=np.uint8)
+    want = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = ue4m3_to_f64(codes)
+    fin = np.isfinite(want)
+    assert np.array_equal(got[fin], want[fin]) and np.all(np.isnan(got[~fin]))
+    assert np.array_equal(ue4m3_to_f64(codes[:127] | 0x80), got[:127])
+
+
+def check_nvfp4_golden(dequant_nvfp4):
+    """Hand-decoded two-block row stored in tests/golden/nvfp4_two_blocks.json."""
+    with open(os.path.join(GOLDEN, "nvfp4_two_blocks.json")) as f:
+        g = json.load(f)
+    got = dequant_nvfp4(np.array([g["packed"]], np.uint8), np.array([g["scales"]], np.uint8))[0]
+    want = np.array(g["values"])
+    assert np.array_equal(got, want) and np.array_equal(np.signbit(got), np.signbit(want))
+
+
+def check_nvfp4_products_exact():
+    """Every E2M1 x UE4M3 product (finite scales) is exactly a bf16 and an f16
+    value: a kernel that dequantises to bf16 loses nothing."""
+    vals = np.array(OCP_E2M1 + [-x for x in OCP_E2M1])
+    sc = torch.arange(127, dtype=torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    prod = (vals[:, None] * sc[None, :]).ravel()
+    t = torch.from_numpy(prod)
+    assert torch.equal(t.to(torch.bfloat16).to(torch.float64), t)
+    assert torch.equal(t.to(torch.float16).to(torch.float64), t)
+
+
+def _table_dequant(packed, scales):
+    """Test-side NVFP4 decoder by table lookup (independent of the oracle's)."""
+    tab = OCP_E2M1 + [-x for x in OCP_E2M1]
+    e4m3 = torch.arange(256, dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn).to(torch.float64)
+    out = []
+    for i, byte in enumerate(packed):
+        s = float(e4m3[int(scales[(2 * i) // 16]) & 0x7F])
+        out += [tab[byte & 0xF] * s, tab[byte >> 4] * s]
+    return out
+
+
+def check_nvfp4_decode_brute_force(reference_decode):
+    """A tiny NVFP4 decode (2 requests, causal s_q 2, d_qk = d_v = 512) against
+    50-digit brute force over values decoded by table lookup."""
+    import dataclasses
+    from workloads import mla_workloads as W
+    w = dataclasses.replace(W.get_workload("tiny"), kv="nvfp4", batch=2, seqlens=[3, 2], s_q=2, h_q=2,
+                            causal=True, scale=512 ** -0.5, seed=41)
+    inp = W.make_inputs(w)
+    out, lse = reference_decode(inp)
+    bt = inp.block_table.numpy()
+    for b, L in enumerate([3, 2]):
+        rows = []
+        for t in range(L):
+            pg, sl = bt[b, t // PAGE], t % PAGE
+            rows.append(_table_dequant(inp.kcache[pg, sl].tolist(), inp.kv_scale[pg, sl].tolist()))
+        for i in range(2):
+            n = L - 2 + i + 1
+            qs = [_table_dequant(inp.q[b, i, h].tolist(), inp.q_scale[b, i, h].tolist()) for h in range(2)]
+            eo, el = _mp_attend(qs, rows[:n], 512 ** -0.5, 512)
+            _close(out[b, i], eo, 1e-13)
+            _close(lse[b, i], el, 1e-13)

@@ -205,3 +205,45 @@ def test_sink_in_every_split_caught():
         op = o_parts * np.exp(lse_parts - lp)[..., None]
         return real_combine(op, lp)
     assert _fails(C.check_sink_reductions, O.decode_dense, O.decode_sparse, O.attend, per_part)
+
+
+# ---------------------------------------------------------------- NVFP4
+real_dequant_nvfp4 = O.dequant_nvfp4
+
+
+def _nvfp4_nibbles_swapped(packed, scales):
+    pk = np.asarray(packed, dtype=np.uint8)
+    return real_dequant_nvfp4(((pk & 0xF) << 4) | (pk >> 4), scales)
+
+
+def _nvfp4_block32(packed, scales):
+    sc = np.asarray(scales, dtype=np.uint8)
+    sc2 = np.repeat(sc[..., 0::2], 2, axis=-1)        # one scale per 32 values
+    return real_dequant_nvfp4(packed, sc2)
+
+
+def _nvfp4_scale_e8m0(packed, scales):
+    pk = np.asarray(packed, dtype=np.uint8)
+    codes = np.stack([pk & 0xF, pk >> 4], axis=-1).reshape(*pk.shape[:-1], 2 * pk.shape[-1])
+    sc = np.exp2(np.asarray(scales, dtype=np.float64) - 127.0)
+    return O.e2m1_to_f64(codes) * np.repeat(sc, 16, axis=-1)
+
+
+def _e2m1_bias0(codes):
+    c = np.asarray(codes).astype(np.int64) & 0xF
+    e, m = (c >> 1) & 3, c & 1
+    mag = np.where(e == 0, 0.5 * m, np.exp2(e * 1.0) * (1.0 + 0.5 * m))
+    return np.where(c & 8, -mag, mag)
+
+
+@pytest.mark.parametrize("mutant", [_nvfp4_nibbles_swapped, _nvfp4_block32, _nvfp4_scale_e8m0],
+                         ids=lambda f: f.__name__)
+def test_nvfp4_layout_mutants_caught(mutant, monkeypatch):
+    caught = _fails(C.check_nvfp4_golden, mutant)
+    monkeypatch.setattr(O, "dequant_nvfp4", mutant)
+    caught = caught or _fails(C.check_nvfp4_decode_brute_force, O.reference_decode)
+    assert caught
+
+
+def test_e2m1_bias_mistake_caught():
+    assert _fails(C.check_e2m1, _e2m1_bias0)

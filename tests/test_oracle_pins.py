@@ -76,3 +76,23 @@ def test_sink_as_extra_key():
 
 def test_sink_reductions():
     C.check_sink_reductions(O.decode_dense, O.decode_sparse, O.attend, O.combine)
+
+
+def test_e2m1_all_codes():
+    C.check_e2m1(O.e2m1_to_f64)
+
+
+def test_ue4m3_all_codes():
+    C.check_ue4m3(O.ue4m3_to_f64)
+
+
+def test_nvfp4_golden_row():
+    C.check_nvfp4_golden(O.dequant_nvfp4)
+
+
+def test_nvfp4_products_exact_in_bf16():
+    C.check_nvfp4_products_exact()
+
+
+def test_nvfp4_decode_brute_force():
+    C.check_nvfp4_decode_brute_force(O.reference_decode)

@@ -40,6 +40,9 @@ D_ROPE = D_QK - D_V
 FP8_TILE = 128
 FP8_RECORD_BYTES = D_V + 4 * (D_V // FP8_TILE) + 2 * D_ROPE  # 656
 E4M3_MAX = 448.0
+NVFP4_D = 512                 # NVFP4 rows: 512 values, the whole row is K and V
+NVFP4_BLOCK = 16              # values per UE4M3 scale
+E2M1_MAGNITUDES = (0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0)   # codes 0..7 (OCP MX FP4)
 
 
 @dataclass
@@ -50,7 +53,7 @@ class Workload:
     h_q: int
     seqlens: list
     causal: bool
-    kv: str = "bf16"            # "bf16" | "fp8"
+    kv: str = "bf16"            # "bf16" | "fp8" | "nvfp4"
     topk: int = 0               # >0: token-sparse decode
     neg_frac: float = 0.0       # fraction of index slots set to -1
     scale: float = 1.0 / math.sqrt(D_QK)
@@ -60,6 +63,10 @@ class Workload:
     @property
     def rows(self) -> int:
         return self.s_q * self.h_q
+
+    @property
+    def d_qk(self) -> int:
+        return NVFP4_D if self.kv == "nvfp4" else D_QK
 
 
 def _mtp_seqlens(seed: int):
@@ -137,6 +144,8 @@ class DecodeInputs:
     indices: Optional[torch.Tensor] = None   # [B, s_q, topk] int32
     extra: dict = field(default_factory=dict)
     sink: Optional[torch.Tensor] = None      # [h_q] fp32 per-head attention-sink logits
+    q_scale: Optional[torch.Tensor] = None   # nvfp4: uint8 [B, s_q, h_q, 32] UE4M3 block scales
+    kv_scale: Optional[torch.Tensor] = None  # nvfp4: uint8 [P, 64, 32] UE4M3 block scales
 
     @property
     def num_pages(self) -> int:
@@ -164,6 +173,29 @@ def quantize_fp8_records(src: torch.Tensor) -> torch.Tensor:
     return rec
 
 
+def quantize_nvfp4(src: torch.Tensor):
+    """fp32 [..., 512] -> (uint8 [..., 256] packed E2M1, uint8 [..., 32] UE4M3).
+
+    Per block of 16 values: scale = e4m3(amax / 6) by torch's fp8 conversion
+    (round to nearest even; 0 when amax == 0); code = the E2M1 magnitude
+    nearest |x| / scale (ties to the smaller magnitude, saturating at 6) with
+    the sign of x; element 2i in the low nibble of byte i. This is data
+    preparation: the decode path only reads codes and scales.
+    """
+    shp = src.shape
+    blk = src.reshape(*shp[:-1], shp[-1] // NVFP4_BLOCK, NVFP4_BLOCK).to(torch.float32)
+    amax = blk.abs().amax(dim=-1)
+    sc8 = (amax / 6.0).to(torch.float8_e4m3fn)
+    sc = sc8.to(torch.float32)
+    y = torch.where(sc[..., None] > 0, blk / torch.where(sc > 0, sc, torch.ones_like(sc))[..., None],
+                    torch.zeros_like(blk))
+    mags = torch.tensor(E2M1_MAGNITUDES, dtype=torch.float32)
+    idx = (y.abs()[..., None] - mags).abs().argmin(dim=-1)           # first minimum: smaller magnitude
+    codes = (idx | torch.where(y < 0, 8, 0)).to(torch.uint8).reshape(*shp[:-1], shp[-1])
+    packed = (codes[..., 0::2] | (codes[..., 1::2] << 4)).contiguous()
+    return packed, sc8.view(torch.uint8).contiguous()
+
+
 def make_inputs(w: Workload, *, poison_tail: bool = False, extra_pages: int = 0,
                 seqlens_override=None) -> DecodeInputs:
     """Build the seeded host-side inputs of one workload.
@@ -176,7 +208,11 @@ def make_inputs(w: Workload, *, poison_tail: bool = False, extra_pages: int = 0,
     seqlens = list(seqlens_override) if seqlens_override is not None else list(w.seqlens)
     B = w.batch
     assert len(seqlens) == B
-    q = _normal_bf16(rng, (B, w.s_q, w.h_q, D_QK))
+    q_scale = kv_scale = None
+    if w.kv == "nvfp4":
+        q, q_scale = quantize_nvfp4(_normal_f32(rng, (B, w.s_q, w.h_q, NVFP4_D)))
+    else:
+        q = _normal_bf16(rng, (B, w.s_q, w.h_q, D_QK))
     npages = [(L + PAGE - 1) // PAGE for L in seqlens]
     P_used = int(sum(npages))
     P = P_used + extra_pages
@@ -187,7 +223,15 @@ def make_inputs(w: Workload, *, poison_tail: bool = False, extra_pages: int = 0,
     for b in range(B):
         bt[b, :npages[b]] = perm[off:off + npages[b]]
         off += npages[b]
-    if w.kv == "bf16":
+    if w.kv == "nvfp4":
+        kc, kv_scale = quantize_nvfp4(_normal_f32(rng, (P, PAGE, NVFP4_D)))
+        if poison_tail:   # UE4M3 0x7F is NaN: every value of a poisoned token is NaN
+            for b in range(B):
+                if npages[b] and seqlens[b] % PAGE:
+                    kv_scale[int(bt[b, npages[b] - 1]), seqlens[b] % PAGE:] = 0x7F
+            for p in perm[P_used:]:
+                kv_scale[int(p)] = 0x7F
+    elif w.kv == "bf16":
         kc = _normal_bf16(rng, (P, PAGE, 1, D_QK))
         if poison_tail:
             nan = torch.tensor(float("nan"), dtype=torch.bfloat16)
@@ -221,7 +265,7 @@ def make_inputs(w: Workload, *, poison_tail: bool = False, extra_pages: int = 0,
     return DecodeInputs(
         workload=w, q=q, kcache=kc, block_table=torch.from_numpy(bt),
         cache_seqlens=torch.tensor(seqlens, dtype=torch.int32), indices=idx,
-        extra={"pages_per_request": npages})
+        extra={"pages_per_request": npages}, q_scale=q_scale, kv_scale=kv_scale)
 
 
 def make_sink(h_q: int, seed: int) -> torch.Tensor:
@@ -240,14 +284,16 @@ def with_sink(inp: "DecodeInputs", seed: int = 0) -> "DecodeInputs":
 def algorithmic_work(inp: DecodeInputs) -> dict:
     """FLOPs and bytes the method must do for one decode call.
 
-    FLOPs = 2 * sum over (request, query row, head) of |key set| * (576 + 512),
-    counting only unmasked, non-ignored keys. Bytes = distinct cache rows
-    touched (1152 B bf16 / 656 B fp8) + q + out + lse + block table, seqlens
-    and indices read.
+    FLOPs = 2 * sum over (request, query row, head) of |key set| * (d_qk + 512)
+    (d_qk 576, or 512 for NVFP4 rows), counting only unmasked, non-ignored
+    keys. Bytes = distinct cache rows touched (1152 B bf16 / 656 B fp8 / 288 B
+    nvfp4) + q + out + lse + block table, seqlens and indices read.
     """
     w = inp.workload
     seqlens = inp.cache_seqlens.tolist()
-    row_bytes = 2 * D_QK if w.kv == "bf16" else FP8_RECORD_BYTES
+    row_bytes = {"bf16": 2 * D_QK, "fp8": FP8_RECORD_BYTES, "nvfp4": NVFP4_D // 2 + NVFP4_D // NVFP4_BLOCK}[w.kv]
+    d_qk = w.d_qk
+    q_bytes = 2 * D_QK if w.kv != "nvfp4" else NVFP4_D // 2 + NVFP4_D // NVFP4_BLOCK
     keys = 0
     touched = 0
     if w.topk:
@@ -267,9 +313,9 @@ def algorithmic_work(inp: DecodeInputs) -> dict:
             for i in range(w.s_q):
                 lim = L - w.s_q + i + 1 if w.causal else L
                 keys += max(0, min(L, lim)) * w.h_q
-    flops = 2.0 * keys * (D_QK + D_V)
+    flops = 2.0 * keys * (d_qk + D_V)
     rows = w.batch * w.s_q * w.h_q
-    byts = touched * row_bytes + rows * (2 * D_QK + 2 * D_V + 4)
+    byts = touched * row_bytes + rows * (q_bytes + 2 * D_V + 4)
     if w.topk:
         byts += inp.indices.numel() * 4 + keys // max(1, w.h_q) * 4   # indices + one page lookup each
     else:
@@ -300,4 +346,5 @@ def restrict(inp: DecodeInputs, requests) -> DecodeInputs:
         workload=w, q=inp.q[requests].clone(), kcache=inp.kcache[pages].clone(),
         block_table=torch.from_numpy(new_bt), cache_seqlens=torch.tensor(sub_lens, dtype=torch.int32),
         indices=None if inp.indices is None else inp.indices[requests].clone(),
-        sink=inp.sink)
+        sink=inp.sink, q_scale=None if inp.q_scale is None else inp.q_scale[requests].clone(),
+        kv_scale=None if inp.kv_scale is None else inp.kv_scale[pages].clone())
