@@ -137,7 +137,7 @@ class ClockSampler:
 def workload_config(inp, work):
     w = inp.workload
     cfg = {"workload": f"{w.name}: {w.note}", "batch": w.batch, "s_q": w.s_q, "h_q": w.h_q,
-           "h_kv": 1, "d_qk": 576, "d_v": 512, "page": 64, "kv_cache": w.kv,
+           "h_kv": 1, "d_qk": w.d_qk, "d_v": 512, "page": 64, "kv_cache": w.kv,
            "causal": w.causal, "softmax_scale": w.scale,
            "tokens_cached": int(sum(int(x) for x in inp.cache_seqlens.tolist())),
            "algorithmic_flops": work["flops"], "algorithmic_bytes": work["bytes"],
@@ -238,7 +238,10 @@ def run_gpu(args):
     sl = inp.cache_seqlens.to(dev)
     idx = inp.indices.to(dev) if inp.indices is not None else None
     sink = inp.sink.to(dev) if inp.sink is not None else None
-    runner = M.DecodeRunner(q, kc, bt, sl, softmax_scale=w.scale, causal=w.causal, indices=idx, sink=sink)
+    qs = inp.q_scale.to(dev) if inp.q_scale is not None else None
+    ks = inp.kv_scale.to(dev) if inp.kv_scale is not None else None
+    runner = M.DecodeRunner(q, kc, bt, sl, softmax_scale=w.scale, causal=w.causal, indices=idx, sink=sink,
+                            q_scale=qs, kv_scale=ks)
     # timing variant: the decode kernel alone, then the combine enqueued by the caller
     runner.args.debug_flags = C.MLA_DEBUG_SKIP_COMBINE
     U, R, P = runner.units, runner.rows, runner.parts
@@ -302,9 +305,11 @@ def run_gpu(args):
     bt_h = inp.block_table.pin_memory()
     sl_h = inp.cache_seqlens.pin_memory()
     idx_h = inp.indices.pin_memory() if inp.indices is not None else None
+    qs_h = inp.q_scale.pin_memory() if inp.q_scale is not None else None
     out_h = torch.empty(runner.out.shape, dtype=runner.out.dtype).pin_memory()
     lse_h = torch.empty(runner.lse.shape, dtype=runner.lse.dtype).pin_memory()
-    runner_e2e = M.DecodeRunner(q, kc, bt, sl, softmax_scale=w.scale, causal=w.causal, indices=idx, sink=sink)
+    runner_e2e = M.DecodeRunner(q, kc, bt, sl, softmax_scale=w.scale, causal=w.causal, indices=idx, sink=sink,
+                                q_scale=qs, kv_scale=ks)
 
     def e2e_step():
         q.copy_(q_h, non_blocking=True)
@@ -312,6 +317,8 @@ def run_gpu(args):
         sl.copy_(sl_h, non_blocking=True)
         if idx is not None:
             idx.copy_(idx_h, non_blocking=True)
+        if qs is not None:
+            qs.copy_(qs_h, non_blocking=True)
         runner_e2e.plan(stream)
         runner_e2e.run(stream)
         out_h.copy_(runner_e2e.out, non_blocking=True)
@@ -336,6 +343,8 @@ def run_gpu(args):
     h2d = q_h.numel() * q_h.element_size() + bt_h.numel() * 4 + sl_h.numel() * 4
     if idx_h is not None:
         h2d += idx_h.numel() * 4
+    if qs_h is not None:
+        h2d += qs_h.numel()
     d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * 4
 
     if pg:
@@ -370,7 +379,9 @@ def run_gpu(args):
     value = world * work["flops"] / (ms_step * 1e-3) / 1e12
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16" if w.kv == "bf16" else "fp8-e4m3 cache, bf16 mma",
+            "vs_baseline": None,
+            "dtype": {"bf16": "bf16", "fp8": "fp8-e4m3 cache, bf16 mma",
+                      "nvfp4": "nvfp4 (e2m1 + ue4m3) query and cache, dequantised exactly to bf16 mma"}[w.kv],
             "data": "synthetic", "config": workload_config(inp, work),
             "hbm_gbs": world * work["bytes"] / (ms_step * 1e-3) / 1e9,
             "roofline": roof, "clocks": dict(clocks.summary(), remeasured=remeasured),

@@ -25,6 +25,7 @@ MLA_ERR_DEVICE_TIMEOUT = 5
 MLA_ERR_DEVICE_BOUNDS = 6
 MLA_KV_BF16 = 0
 MLA_KV_FP8_E4M3 = 1
+MLA_KV_NVFP4 = 2
 MLA_DEVICE_STATUS_TIMEOUT = 1
 MLA_DEVICE_STATUS_BOUNDS = 2
 MLA_DEBUG_WITHHOLD_SCORES = 1
@@ -51,7 +52,7 @@ class MlaDecodeArgs(ctypes.Structure):
         ("num_pages", ctypes.c_int), ("block_table_stride", ctypes.c_int), ("num_sm_parts", ctypes.c_int),
         ("softmax_scale", ctypes.c_float), ("causal", ctypes.c_int), ("kv_format", ctypes.c_int),
         ("timeout_ns", ctypes.c_uint64), ("debug_flags", ctypes.c_uint32),
-        ("sink", ctypes.c_void_p),
+        ("sink", ctypes.c_void_p), ("q_scale", ctypes.c_void_p), ("kv_scale", ctypes.c_void_p),
     ]
 
 
@@ -155,7 +156,7 @@ def mla_workspace_size(batch, s_q, h_q, h_kv, topk, num_sm_parts) -> int:
 def make_args(*, q, kcache, block_table, cache_seqlens, tile_md, num_splits, out, lse, workspace,
               batch, s_q, h_q, h_kv, num_pages, num_sm_parts, softmax_scale, causal, kv_format,
               block_table_stride=None, d_qk=576, d_v=512, page_size=64, timeout_ns=0, debug_flags=0,
-              workspace_bytes=None, sink=None) -> MlaDecodeArgs:
+              workspace_bytes=None, sink=None, q_scale=None, kv_scale=None) -> MlaDecodeArgs:
     a = MlaDecodeArgs()
     a.q, a.kcache, a.block_table = _ptr(q), _ptr(kcache), _ptr(block_table)
     a.cache_seqlens, a.tile_md, a.num_splits = _ptr(cache_seqlens), _ptr(tile_md), _ptr(num_splits)
@@ -172,6 +173,8 @@ def make_args(*, q, kcache, block_table, cache_seqlens, tile_md, num_splits, out
     a.timeout_ns = timeout_ns
     a.debug_flags = debug_flags
     a.sink = _ptr(sink)
+    a.q_scale = _ptr(q_scale)
+    a.kv_scale = _ptr(kv_scale)
     return a
 
 

@@ -64,8 +64,12 @@ mla_status_t check_common(const mla_decode_args* a, int topk) {
   if (a->batch <= 0 || a->s_q <= 0 || a->h_q <= 0 || a->h_kv <= 0 || a->num_pages <= 0 ||
       a->block_table_stride <= 0 || a->num_sm_parts <= 0)
     return MLA_ERR_INVALID_ARG;
-  if (a->d_qk != kDqk || a->d_v != kDv || a->page_size != kPage) return MLA_ERR_INVALID_ARG;
-  if (a->kv_format != MLA_KV_BF16 && a->kv_format != MLA_KV_FP8_E4M3) return MLA_ERR_INVALID_ARG;
+  if (a->kv_format != MLA_KV_BF16 && a->kv_format != MLA_KV_FP8_E4M3 && a->kv_format != MLA_KV_NVFP4)
+    return MLA_ERR_INVALID_ARG;
+  const bool nvfp4 = a->kv_format == MLA_KV_NVFP4;
+  if (a->d_qk != (nvfp4 ? kNvfp4D : kDqk) || a->d_v != kDv || a->page_size != kPage) return MLA_ERR_INVALID_ARG;
+  if (nvfp4 && (!a->q_scale || !a->kv_scale || !aligned16(a->kv_scale))) return MLA_ERR_INVALID_ARG;
+  if (nvfp4 && topk > 0) return MLA_ERR_UNSUPPORTED;
   if (!(a->softmax_scale > 0.f) || !std::isfinite(a->softmax_scale)) return MLA_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(a->sink) & 3u) != 0) return MLA_ERR_INVALID_ARG;
   if (a->h_kv != 1) return MLA_ERR_UNSUPPORTED;
@@ -85,17 +89,20 @@ mla_status_t run_decode(const mla_decode_args* a, const int32_t* indices, int to
   const int rows = g.rows;
   const int U = a->batch * g.units_per_req;
   const bool fp8 = a->kv_format == MLA_KV_FP8_E4M3;
-  const int mode = topk > 0 ? (fp8 ? kModeFp8Sparse : kModeSparse) : (fp8 ? kModeFp8 : kModeBf16);
+  const int mode = a->kv_format == MLA_KV_NVFP4 ? kModeNvfp4
+                   : topk > 0                  ? (fp8 ? kModeFp8Sparse : kModeSparse)
+                                               : (fp8 ? kModeFp8 : kModeBf16);
   // Q rows of every unit, and (bf16 paged cache only) the cache as
   // [pages*64 tokens][576 dims]; boxes of 64 x 64 with 128-B swizzle. The FP8
   // and sparse modes read the cache with cp.async and need no cache map.
   CUtensorMap tq, tkv;
+  std::memset(&tq, 0, sizeof(tq));
   std::memset(&tkv, 0, sizeof(tkv));
-  if (!make_map(&tq, a->q, (uint64_t)U * rows, kDqk, kDqk * 2, 64, 64)) return MLA_ERR_CUDA;
+  if (mode != kModeNvfp4 && !make_map(&tq, a->q, (uint64_t)U * rows, kDqk, kDqk * 2, 64, 64)) return MLA_ERR_CUDA;
   const int row_groups = (rows + kRowsPerCta - 1) / kRowsPerCta;
   // more than 64 rows on the BF16 cache (paged or sparse): one CTA pair per
   // part shares each cache tile between the two row halves
-  const bool pair = row_groups == 2 && !mode_fp8(mode);
+  const bool pair = row_groups == 2 && (mode == kModeBf16 || mode == kModeSparse);
   if (mode == kModeBf16 &&
       !make_map(&tkv, a->kcache, (uint64_t)a->num_pages * kPage, kDqk, kDqk * 2, 64, 64))
     return MLA_ERR_CUDA;
@@ -129,6 +136,9 @@ mla_status_t run_decode(const mla_decode_args* a, const int32_t* indices, int to
   p.timeout_ns = a->timeout_ns ? a->timeout_ns : 2000000000ull;
   p.debug_flags = a->debug_flags;
   p.sink = a->sink;
+  p.q_nvfp4 = static_cast<const uint8_t*>(a->q);
+  p.q_scale = static_cast<const uint8_t*>(a->q_scale);
+  p.kv_scale = static_cast<const uint8_t*>(a->kv_scale);
   const int rows_per_cta = rows < kRowsPerCta ? rows : kRowsPerCta;
   const cudaError_t e = pair ? launch_decode_pair(tq, tkv, p, a->num_sm_parts, mode == kModeSparse, stream)
                              : launch_decode(rows_per_cta, mode, tq, tkv, p, a->num_sm_parts, row_groups, stream);

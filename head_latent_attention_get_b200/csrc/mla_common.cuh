@@ -14,6 +14,9 @@ constexpr int kTile = 128;              // tokens per scheduler block / kernel t
 constexpr int kRowsPerCta = 64;         // query rows handled by one CTA
 constexpr int kSchedOverhead = 3;       // fixed cost of a piece, in tiles
 constexpr int kFp8RecordBytes = 656;    // 512 e4m3 + 4 fp32 scales + 64 bf16
+constexpr int kNvfp4D = 512;            // NVFP4 rows: 512 values, K and V
+constexpr int kNvfp4RowBytes = 256;     // packed E2M1, two per byte
+constexpr int kNvfp4ScaleBytes = 32;    // one UE4M3 per 16 values
 constexpr size_t kWsHeaderBytes = 256;  // device status word lives at offset 0
 
 __host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }

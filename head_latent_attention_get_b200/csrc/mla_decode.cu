@@ -51,6 +51,10 @@ constexpr int kTmemS = 256;            // S buffers at columns 256 and 384
 constexpr float kRescaleLog2 = 8.0f;   // rescale O only when the max grows by > 2^8
 static_assert(kLag < kNK && kLag < kNV, "a gather group must retire a slot before reusing it");
 
+// K slices of 64 dims per tile: 576-dim rows (512 latent + 64 RoPE) or the
+// 512-value NVFP4 rows.
+__host__ __device__ constexpr int k_slices(int mode) { return mode == kModeNvfp4 ? 8 : 9; }
+
 template <int NR>
 struct Smem {
   static constexpr int q = 0;
@@ -126,7 +130,54 @@ template <int MODE, bool KGROUP>
 __device__ __forceinline__ void retire_slot(const GatherRing& g, int seq, int lw, int t) {
   const int slot = seq % g.nslots;
   uint8_t* s = g.base + slot * kSlot;
-  if (mode_fp8(MODE)) {
+  if (MODE == kModeNvfp4) {
+    __syncwarp();  // every lane's copies of this slot are complete and visible
+    if (KGROUP) {  // slice j: codes in bytes [0,32), the 16-byte scale chunk 16*(j/4).. in [32,48) of each row
+      const int j = seq % 8;
+      uint2 cw[4];
+      uint32_t sb[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = 32 * lw + 8 * i + (t >> 2), cc = t & 3;  // values 16cc..16cc+15 of the slice
+        cw[i] = *reinterpret_cast<const uint2*>(s + r * 128 + 8 * cc);
+        sb[i] = s[r * 128 + 32 + 4 * (j & 3) + cc];
+      }
+      __syncwarp();
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = 32 * lw + 8 * i + (t >> 2), cc = t & 3;
+        uint4 lo, hi;
+        dequant_nvfp4_16(cw[i], sb[i], lo, hi);
+        *reinterpret_cast<uint4*>(sw128(s, r, 2 * cc)) = lo;
+        *reinterpret_cast<uint4*>(sw128(s, r, 2 * cc + 1)) = hi;
+      }
+    } else {  // V slot: codes (64 B) and the scale chunk 16*(m/2).. in the half-0 row
+      const int m = (seq >> 1) & 3;
+      uint4 cw[2];
+      uint32_t sb[2][2];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int r = 16 * lw + 8 * i + (t >> 2), c4 = t & 3;  // values 32c4..32c4+31 of the 128
+        cw[i] = *reinterpret_cast<const uint4*>(s + r * 128 + 16 * c4);
+        sb[i][0] = s[r * 128 + 64 + 8 * (m & 1) + 2 * c4];
+        sb[i][1] = s[r * 128 + 64 + 8 * (m & 1) + 2 * c4 + 1];
+      }
+      __syncwarp();
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int r = 16 * lw + 8 * i + (t >> 2), c4 = t & 3;
+        uint8_t* half = s + (c4 >> 1) * 8192;
+        const int c0 = 4 * (c4 & 1);
+        uint4 lo, hi;
+        dequant_nvfp4_16(make_uint2(cw[i].x, cw[i].y), sb[i][0], lo, hi);
+        *reinterpret_cast<uint4*>(sw128(half, r, c0)) = lo;
+        *reinterpret_cast<uint4*>(sw128(half, r, c0 + 1)) = hi;
+        dequant_nvfp4_16(make_uint2(cw[i].z, cw[i].w), sb[i][1], lo, hi);
+        *reinterpret_cast<uint4*>(sw128(half, r, c0 + 2)) = lo;
+        *reinterpret_cast<uint4*>(sw128(half, r, c0 + 3)) = hi;
+      }
+    }
+  } else if (mode_fp8(MODE)) {
     __syncwarp();  // every lane's copies of this slot are complete and visible
     if (KGROUP) {
       const int j = seq % 9;
@@ -197,7 +248,8 @@ __device__ __forceinline__ const uint8_t* gather_src(const DecodeParams& p, int 
   int pg = page_of(p, req, 2 * k + (tt >> 6), npg);
   if (pg < 0) pg = page_of(p, req, 2 * k, npg);  // half tile: page A again (keys masked, values zero-filled later)
   ok = 16u;
-  return p.kcache_fp8 + ((size_t)pg * kPage + (tt & 63)) * kFp8RecordBytes;
+  const size_t rb = MODE == kModeNvfp4 ? (size_t)kNvfp4RowBytes : (size_t)kFp8RecordBytes;
+  return p.kcache_fp8 + ((size_t)pg * kPage + (tt & 63)) * rb;
 }
 
 template <int MODE, bool KGROUP>
@@ -223,12 +275,34 @@ __device__ void gather_group(const DecodeParams& p, Ctrl* c, PieceIter& it, cons
         srcV0 = gather_src<MODE, KGROUP>(p, unit, req, npg, k, 16 * lw + (t & 15), ok0);
         srcV1 = gather_src<MODE, KGROUP>(p, unit, req, npg, k, 64 + 16 * lw + (t & 15), ok1);
       }
-      const int slots_per_tile = KGROUP ? 9 : 8;
+      const int slots_per_tile = KGROUP ? k_slices(MODE) : 8;
       for (int j = 0; j < slots_per_tile; ++j, ++seq) {
         const int slot = seq % g.nslots;
         uint8_t* s = g.base + slot * kSlot;
         if (!timed_wait(c, &g.empty[slot], ((seq / g.nslots) & 1) ^ 1, p)) { stop = true; break; }
-        if (KGROUP) {
+        if (MODE == kModeNvfp4) {
+          // row pointers: codes (256 B per row) and scales (32 B per row, the
+          // row's byte offset / 8 into the scale array)
+          if (KGROUP) {  // slice j: 32 code bytes (2 lanes per row) + a 16-byte scale chunk
+            const uint8_t* srcS = p.kv_scale + ((srcK - p.kcache_fp8) >> 3);
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+              const int r = 16 * i + (t >> 1), ch = t & 1;
+              cp_async16(s + (32 * lw + r) * 128 + 16 * ch, shfl_ptr(srcK, r) + 32 * j + 16 * ch, 16u);
+            }
+            cp_async16(s + (32 * lw + t) * 128 + 32, srcS + 16 * (j >> 2), 16u);
+          } else {  // V slot j: 64 code bytes of value group m (4 lanes per row) + a scale chunk
+            const int m = j >> 1;
+            const uint8_t* sv = (j & 1) ? srcV1 : srcV0;
+            const uint8_t* srcS = p.kv_scale + ((sv - p.kcache_fp8) >> 3);
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+              const int r = 8 * i + (t >> 2), ch = t & 3;
+              cp_async16(s + (16 * lw + r) * 128 + 16 * ch, shfl_ptr(sv, r) + 64 * m + 16 * ch, 16u);
+            }
+            if (t < 16) cp_async16(s + (16 * lw + t) * 128 + 64, srcS + 16 * (m >> 1), 16u);
+          }
+        } else if (KGROUP) {
           if (MODE == kModeSparse || j == 8) {  // bf16 128-B row slice: 8 lanes per row
             const int off = MODE == kModeSparse ? 128 * j : 528;
 #pragma unroll
@@ -322,7 +396,7 @@ __global__ void __launch_bounds__(MODE == kModeBf16 ? 256 : 256 + 2 * kGatherThr
     c->rescale_flag[1] = 0;
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) {
+  if (warp == 0 && lane == 0 && MODE != kModeNvfp4) {
     tma_prefetch_desc(&tm_q);
     if (MODE == kModeBf16) tma_prefetch_desc(&tm_kv);  // encoded only for the bf16 paged cache
   }
@@ -344,6 +418,40 @@ __global__ void __launch_bounds__(MODE == kModeBf16 ? 256 : 256 + 2 * kGatherThr
     int kc = 0, pi = 0, q_issued = 0;
     bool stop = false;
     while (!stop && it.next(pc)) {
+      if (MODE == kModeNvfp4) {
+        // Q rows dequantised by this warp: lane l converts value block l
+        // (dims 16l..16l+15) of each row into box l/4, chunks 2(l%4), 2(l%4)+1;
+        // rows past this CTA's rows are zero
+        if (lane == 0 && !timed_wait(c, &c->q_empty, (pi & 1) ^ 1, p)) stop = true;
+        stop = __shfl_sync(0xffffffffu, stop ? 1 : 0, 0) != 0;
+        if (stop) break;
+        const size_t qrow0 = (size_t)pc.unit * p.rows + row0;
+        uint8_t* box = sQ + (lane >> 2) * 8192;
+#pragma unroll 1
+        for (int r0 = 0; r0 < kRowsPerCta; r0 += 8) {
+          uint2 cw[8];
+          uint32_t sb[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const bool live = r0 + i < rows_here;
+            const size_t qr = qrow0 + (live ? r0 + i : 0);
+            cw[i] = live ? *reinterpret_cast<const uint2*>(p.q_nvfp4 + qr * kNvfp4RowBytes + 8 * lane) : make_uint2(0, 0);
+            sb[i] = live ? p.q_scale[qr * kNvfp4ScaleBytes + lane] : 0u;
+          }
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            uint4 lo, hi;
+            dequant_nvfp4_16(cw[i], sb[i], lo, hi);
+            *reinterpret_cast<uint4*>(sw128(box, r0 + i, 2 * (lane & 3))) = lo;
+            *reinterpret_cast<uint4*>(sw128(box, r0 + i, 2 * (lane & 3) + 1)) = hi;
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&c->q_full);
+        ++pi;
+        continue;
+      }
       if (lane == 0) {
         if (!timed_wait(c, &c->q_empty, (pi & 1) ^ 1, p)) {
           stop = true;
@@ -374,7 +482,7 @@ __global__ void __launch_bounds__(MODE == kModeBf16 ? 256 : 256 + 2 * kGatherThr
       stop = __shfl_sync(0xffffffffu, stop ? 1 : 0, 0) != 0;
       ++pi;
     }
-    if (lane == 0) {
+    if (lane == 0 && MODE != kModeNvfp4) {
       if (q_issued > 0) mbar_wait(&c->q_full, (uint32_t)((q_issued - 1) & 1), p.timeout_ns);
       if (MODE == kModeBf16) drain_issued(c->k_full, kNK, kc, p.timeout_ns);
     }
@@ -428,7 +536,7 @@ __global__ void __launch_bounds__(MODE == kModeBf16 ? 256 : 256 + 2 * kGatherThr
           if (!timed_wait(c, &c->s_empty[b], ((gt >> 1) & 1) ^ 1, p)) { stop = true; }
           tc_fence_after();
           const uint32_t d = tmem + kTmemS + 128 * b;
-          for (int j = 0; j < 9 && !stop; ++j, ++kc) {
+          for (int j = 0; j < k_slices(MODE) && !stop; ++j, ++kc) {
             const int slot = kc % kNK;
             if (!timed_wait(c, &c->k_full[slot], (kc / kNK) & 1, p)) { stop = true; break; }
             tc_fence_after();
@@ -717,6 +825,7 @@ cudaError_t launch_decode(int rows_per_cta, int mode, const CUtensorMap& tq, con
   if (mode == kModeBf16) return launch_one<NRV, kModeBf16>(tq, tkv, p, parts, row_groups, stream); \
   if (mode == kModeFp8) return launch_one<NRV, kModeFp8>(tq, tkv, p, parts, row_groups, stream);   \
   if (mode == kModeSparse) return launch_one<NRV, kModeSparse>(tq, tkv, p, parts, row_groups, stream); \
+  if (mode == kModeNvfp4) return launch_one<NRV, kModeNvfp4>(tq, tkv, p, parts, row_groups, stream);   \
   return launch_one<NRV, kModeFp8Sparse>(tq, tkv, p, parts, row_groups, stream);
   // <= 16 rows run in the 32-row kernel: the extra P^T rows are written as
   // zeros and their output rows are never stored

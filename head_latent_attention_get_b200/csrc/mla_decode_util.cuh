@@ -3,6 +3,7 @@
 // and 128-byte-swizzle addressing.
 #pragma once
 #include <cuda_bf16.h>
+#include <cuda_fp4.h>
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
@@ -133,6 +134,28 @@ __device__ __forceinline__ void dequant16(const uint4 raw, float s, uint4& lo, u
       const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
       const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
       o[2 * i + h] = pack_bf16x2(f.x * s, f.y * s);
+    }
+  }
+  lo = make_uint4(o[0], o[1], o[2], o[3]);
+  hi = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+// NVFP4: 8 bytes of packed E2M1 (16 values, element 2i in the low nibble of
+// byte i) and their UE4M3 scale -> 16 bf16 (two 16-byte chunks). Every
+// E2M1 x UE4M3 product is exact in f16 and in bf16, so the f16 product and
+// the conversions lose nothing.
+__device__ __forceinline__ void dequant_nvfp4_16(const uint2 raw, uint32_t scale_byte, uint4& lo, uint4& hi) {
+  const __half_raw sr = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)(scale_byte & 0x7Fu), __NV_E4M3);
+  const __half2 s2 = __half2half2(*reinterpret_cast<const __half*>(&sr));
+  const uint32_t w[2] = {raw.x, raw.y};
+  uint32_t o[8];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const __half2_raw hr = __nv_cvt_fp4x2_to_halfraw2((__nv_fp4x2_storage_t)((w[i] >> (8 * b)) & 0xFFu), __NV_E2M1);
+      const float2 f = __half22float2(__hmul2(*reinterpret_cast<const __half2*>(&hr), s2));
+      o[4 * i + b] = pack_bf16x2(f.x, f.y);
     }
   }
   lo = make_uint4(o[0], o[1], o[2], o[3]);

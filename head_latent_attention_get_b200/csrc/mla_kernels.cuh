@@ -8,8 +8,8 @@
 namespace mla {
 
 // Cache format x key-set kind: BF16 paged, FP8 paged, BF16 token-sparse,
-// FP8 token-sparse.
-enum KvMode : int { kModeBf16 = 0, kModeFp8 = 1, kModeSparse = 2, kModeFp8Sparse = 3 };
+// FP8 token-sparse, NVFP4 paged (512-value rows, NVFP4 query).
+enum KvMode : int { kModeBf16 = 0, kModeFp8 = 1, kModeSparse = 2, kModeFp8Sparse = 3, kModeNvfp4 = 4 };
 __host__ __device__ constexpr bool mode_fp8(int mode) { return mode == kModeFp8 || mode == kModeFp8Sparse; }
 __host__ __device__ constexpr bool mode_sparse(int mode) { return mode == kModeSparse || mode == kModeFp8Sparse; }
 
@@ -33,6 +33,9 @@ struct DecodeParams {
   uint64_t timeout_ns;
   uint32_t debug_flags;
   const float* sink;                        // per-head sink logits [h_q], or null
+  const uint8_t* q_nvfp4;                   // NVFP4 mode: packed E2M1 query rows [units*rows][256]
+  const uint8_t* q_scale;                   // NVFP4 mode: UE4M3 query scales [units*rows][32]
+  const uint8_t* kv_scale;                  // NVFP4 mode: UE4M3 cache scales [pages*64][32]
 };
 
 #ifdef __CUDACC__

@@ -15,13 +15,23 @@ from . import _capi as C
 
 class DecodeRunner:
     def __init__(self, q, kcache, block_table, cache_seqlens, *, softmax_scale, causal=False,
-                 indices=None, num_sm_parts=None, timeout_ns=0, debug_flags=0, sink=None):
+                 indices=None, num_sm_parts=None, timeout_ns=0, debug_flags=0, sink=None, q_scale=None,
+                 kv_scale=None):
+        """q bf16 [B, s_q, h_q, 576] with a bf16 or FP8-record cache, or (NVFP4)
+        packed uint8 [B, s_q, h_q, 256] with q_scale/kv_scale and a packed
+        uint8 [pages, 64, 256] cache."""
         dev = q.device
         assert dev.type == "cuda", "the decode path runs on a CUDA device only"
         self.batch, self.s_q, self.h_q, d = q.shape
-        assert d == 576
         self.topk = int(indices.shape[-1]) if indices is not None else 0
-        self.kv_format = C.MLA_KV_BF16 if kcache.dtype == torch.bfloat16 else C.MLA_KV_FP8_E4M3
+        if q.dtype == torch.uint8:
+            assert d == 256 and kcache.shape[-1] == 256 and q_scale is not None and kv_scale is not None
+            self.kv_format, d_qk = C.MLA_KV_NVFP4, 512
+        else:
+            assert d == 576
+            self.kv_format = C.MLA_KV_BF16 if kcache.dtype == torch.bfloat16 else C.MLA_KV_FP8_E4M3
+            d_qk = 576
+        self.q_scale, self.kv_scale = q_scale, kv_scale
         upr, self.rows = C.mla_decode_geometry(self.s_q, self.h_q, 1, self.topk)
         self.units = self.batch * upr
         self.parts = num_sm_parts or C.mla_get_num_sm_parts(dev.index or 0, self.s_q, self.h_q, 1, self.topk)
@@ -43,7 +53,7 @@ class DecodeRunner:
             workspace=self.workspace, batch=self.batch, s_q=self.s_q, h_q=self.h_q, h_kv=1,
             num_pages=kcache.shape[0], num_sm_parts=self.parts, softmax_scale=softmax_scale,
             causal=causal, kv_format=self.kv_format, timeout_ns=timeout_ns, debug_flags=debug_flags,
-            sink=sink)
+            sink=sink, d_qk=d_qk, q_scale=q_scale, kv_scale=kv_scale)
 
     def plan(self, stream=None):
         C.mla_get_metadata(self.cache_seqlens, self.batch, self.s_q, self.h_q, 1, self.topk, self.parts,

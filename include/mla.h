@@ -78,7 +78,17 @@ enum {
    *   [528,656) 64 bf16 RoPE dims
    * dequantised value = bf16_rne(fp32(e4m3) * scale), product rounded to
    * nearest in fp32; the RoPE dims are used as stored. */
-  MLA_KV_FP8_E4M3 = 1
+  MLA_KV_FP8_E4M3 = 1,
+  /* NVFP4 rows of 512 values that are both K and V (d_qk = d_v = 512; the
+   * FlashInfer page's nvfp4_mla_decode README, section 2): the cache is
+   * uint8 [num_pages, 64, 256] packed E2M1 (element 2i in the low nibble of
+   * byte i, 2i+1 in the high nibble) with UE4M3 scales uint8 [num_pages, 64,
+   * 32] in mla_decode_args.kv_scale, scale byte j for elements [16j, 16j+16);
+   * the query is packed the same way, uint8 [batch, s_q, h_q, 256], with
+   * scales [batch, s_q, h_q, 32] in q_scale. value = e2m1 * ue4m3 (UE4M3:
+   * E4M3 without a sign; bit 7 is ignored), exact in bf16, which the tensor
+   * cores then use. Paged decoding only. */
+  MLA_KV_NVFP4 = 2
 };
 
 /* Bits of the device status word kept at the start of the workspace. */
@@ -174,7 +184,8 @@ mla_status_t mla_get_metadata_host(const int32_t* cache_seqlens, int batch, int 
 size_t mla_workspace_size(int batch, int s_q, int h_q, int h_kv, int topk, int num_sm_parts);
 
 typedef struct {
-  const void* q;                /* device bf16 [batch, s_q, h_q, 576], 16-B aligned */
+  const void* q;                /* device bf16 [batch, s_q, h_q, 576], 16-B aligned
+                                   (MLA_KV_NVFP4: uint8 [batch, s_q, h_q, 256]) */
   const void* kcache;           /* device, format per kv_format, 16-B aligned */
   const int32_t* block_table;   /* device int32 [batch, block_table_stride]; entry
                                    j of row b = physical page of tokens [64j, 64j+64) */
@@ -186,14 +197,14 @@ typedef struct {
   void* workspace;              /* device, >= mla_workspace_size(...) bytes */
   size_t workspace_bytes;
   int batch, s_q, h_q, h_kv;
-  int d_qk, d_v;                /* must be 576 and 512 */
+  int d_qk, d_v;                /* must be 576 (512 for MLA_KV_NVFP4) and 512 */
   int page_size;                /* must be 64 */
   int num_pages;                /* physical pages in kcache */
   int block_table_stride;       /* int32 elements between block-table rows */
   int num_sm_parts;             /* the value passed to mla_get_metadata */
   float softmax_scale;          /* multiplies q.k before the softmax */
   int causal;                   /* nonzero: causal mask inside the s_q block */
-  int kv_format;                /* MLA_KV_BF16 or MLA_KV_FP8_E4M3 */
+  int kv_format;                /* MLA_KV_BF16, MLA_KV_FP8_E4M3 or MLA_KV_NVFP4 */
   uint64_t timeout_ns;          /* limit of every device wait; 0 = 2 s */
   uint32_t debug_flags;         /* MLA_DEBUG_* test hooks; 0 normally */
   const float* sink;            /* device fp32 [h_q], 4-B aligned, or NULL: per-head
@@ -206,6 +217,10 @@ typedef struct {
                                      out = sum_t e^(s_t - lse) v_t.
                                    An empty key set then gives out 0, lse = sink[h];
                                    sink[h] = -inf is the same as no sink. */
+  const void* q_scale;          /* MLA_KV_NVFP4 only: device uint8 [batch, s_q, h_q, 32]
+                                   UE4M3 query scales; ignored otherwise */
+  const void* kv_scale;         /* MLA_KV_NVFP4 only: device uint8 [num_pages, 64, 32]
+                                   UE4M3 cache scales, 16-B aligned; ignored otherwise */
 } mla_decode_args;
 
 /* Paged decoding: enqueues the decode kernel and the split combine.
@@ -251,7 +266,7 @@ mla_status_t mla_decode_paged_noalloc(const mla_decode_args* args, mla_stream_t 
  * combination of the pages' sparse-decoding figures). tile_md/num_splits
  * come from mla_get_metadata(..., topk).
  * Errors as for mla_decode_paged; UNSUPPORTED also for h_q/h_kv >
- * MLA_MAX_ROWS. */
+ * MLA_MAX_ROWS and for MLA_KV_NVFP4. */
 mla_status_t mla_decode_sparse(const mla_decode_args* args, const int32_t* indices, int topk,
                                mla_stream_t stream);
 

@@ -41,14 +41,17 @@ def to_device(inp, dev="cuda"):
         q=inp.q.to(dev), kcache=inp.kcache.to(dev), block_table=inp.block_table.to(dev),
         cache_seqlens=inp.cache_seqlens.to(dev),
         indices=None if inp.indices is None else inp.indices.to(dev),
-        sink=None if getattr(inp, "sink", None) is None else inp.sink.to(dev))
+        sink=None if getattr(inp, "sink", None) is None else inp.sink.to(dev),
+        q_scale=None if inp.q_scale is None else inp.q_scale.to(dev),
+        kv_scale=None if inp.kv_scale is None else inp.kv_scale.to(dev))
 
 
 def run_gpu(inp, runner_kwargs=None, dev_inputs=None):
     d = dev_inputs or to_device(inp)
     w = inp.workload
     r = DecodeRunner(d["q"], d["kcache"], d["block_table"], d["cache_seqlens"], softmax_scale=w.scale,
-                     causal=w.causal, indices=d["indices"], sink=d.get("sink"), **(runner_kwargs or {}))
+                     causal=w.causal, indices=d["indices"], sink=d.get("sink"), q_scale=d.get("q_scale"),
+                     kv_scale=d.get("kv_scale"), **(runner_kwargs or {}))
     r.plan()
     out, lse = r.run()
     torch.cuda.synchronize()

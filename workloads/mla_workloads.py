@@ -96,14 +96,17 @@ def named_workloads():
 def extra_workloads():
     """Workloads of the rows built beyond the five (seeds 20265+): six query
     tokens per request at 64 heads (the FlashInfer README's DeepSeek-V4 decode
-    geometry, q_len 6, here on the 576-dim BF16 latent rows), and the
-    token-sparse batch over the FP8 token-record cache."""
+    geometry, q_len 6, here on the 576-dim BF16 latent rows), the token-sparse
+    batch over the FP8 token-record cache, and the DeepSeek-V4 geometry on
+    NVFP4 rows (512 values, query and cache E2M1 + UE4M3)."""
     return [
         Workload("mtp6", 64, 6, 64, [4096] * 64, causal=True, seed=20265,
                  note="q_len 6 x 64 heads (384 rows per request), causal, BF16, seqlen 4096"),
         Workload("fp8_sparse", 32, 1, 128, [32768] * 32, causal=False, kv="fp8", topk=2048,
                  neg_frac=0.05, seed=20266,
                  note="token-sparse FP8-record decode, 32768-token caches, topk 2048, 5% -1"),
+        Workload("nvfp4", 32, 6, 64, [8192] * 32, causal=True, kv="nvfp4", scale=512 ** -0.5, seed=20267,
+                 note="NVFP4 512-value rows (K = V) and query, q_len 6 x 64 heads, causal, seqlen 8192"),
     ]
 
 
