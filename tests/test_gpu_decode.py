@@ -22,11 +22,13 @@ def _dense(name="tiny", **over):
 # ------------------------------------------------------------------ scheduler
 @pytest.mark.parametrize("lens,s_q,h_q,topk", [
     ([70, 129], 1, 16, 0), ([4096] * 64, 1, 128, 0), ([0, 5, 0, 300, 9000], 2, 16, 0),
-    (list(range(0, 30000, 97)), 1, 64, 0), ([32768] * 32, 1, 128, 2048), ([100] * 5, 2, 32, 128)])
+    (list(range(0, 30000, 97)), 1, 64, 0), ([32768] * 32, 1, 128, 2048), ([100] * 5, 2, 32, 128),
+    ([(37 * i) % 5000 for i in range(13000)], 1, 16, 0),      # more units than the shared-memory prefix holds
+    ([4096] * 64, 6, 64, 0)])                                 # three row-block units per request
 def test_metadata_device_matches_host_twin(lens, s_q, h_q, topk):
     B = len(lens)
     parts = M.mla_get_num_sm_parts(0, s_q, h_q, 1, topk)
-    U = B * s_q if topk else B
+    U = B * M.mla_decode_geometry(s_q, h_q, 1, topk)[0]
     md_h = np.zeros(parts * 8, np.int32)
     ns_h = np.zeros(U + 1, np.int32)
     lens_np = np.asarray(lens, np.int32)
@@ -36,7 +38,7 @@ def test_metadata_device_matches_host_twin(lens, s_q, h_q, topk):
     M.mla_get_metadata(torch.from_numpy(lens_np).cuda(), B, s_q, h_q, 1, topk, parts, md_d, ns_d)
     torch.cuda.synchronize()
     assert np.array_equal(md_d.cpu().numpy(), md_h) and np.array_equal(ns_d.cpu().numpy(), ns_h)
-    S.check_schedule(md_h, ns_h, lens, B, s_q, topk, parts)
+    S.check_schedule(md_h, ns_h, lens, B, s_q, topk, parts, h_q=h_q)
 
 
 # ------------------------------------------------------------------ combine
