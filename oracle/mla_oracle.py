@@ -40,7 +40,7 @@ Passages followed:
   * DeepSeek MLA geometry (FlashMLA-ETAP summary, limitations paragraph): 576
     head dimension; the value part is the first 512 dims (dv = 512).
 
-Readings where the pages are silent (listed in the design doc as well):
+Readings where the pages are silent:
   * sparse indices are logical token positions of request b, resolved through
     the block table; valid range [0, seqlen_b); any other value except -1 is
     ignored and reported as out of range; duplicates count twice.
