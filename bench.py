@@ -210,22 +210,47 @@ def run_reference(args):
     return 0
 
 
+# ----------------------------------------------------------------------------- ranks
+def init_ranks(device=None, backend="nccl"):
+    """(world, rank, local rank, process group module or None) from the
+    torchrun environment; one process per GPU, a short collective timeout so
+    that ranks waiting on a lost peer end with an error."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        kw = {"device_id": device} if backend == "nccl" and device is not None else {}
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
+        pg = dist
+    return world, rank, local, pg
+
+
+def max_over_ranks(pg, x: float, device) -> float:
+    """The largest of every rank's x (a time: the job is as slow as its slowest rank)."""
+    if pg is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(world: int, flops_per_rank: float, ms: float) -> float:
+    """Whole-job throughput: every rank decodes its own replica of the workload."""
+    return world * flops_per_rank / (ms * 1e-3) / 1e12
+
+
 # ----------------------------------------------------------------------------- GPU path
 def run_gpu(args):
     import head_latent_attention_get_b200 as M
     from head_latent_attention_get_b200 import _capi as C
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    pg = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-        pg = dist
+    world, rank, local, pg = init_ranks(dev, "nccl")
 
     inp = W.make_inputs(W.get_workload(args.workload))
     if args.sink:
@@ -294,11 +319,7 @@ def run_gpu(args):
     meta_ms = [e[0].elapsed_time(e[1]) for e in evs]
     dec_ms = [e[1].elapsed_time(e[2]) for e in evs]
     comb_ms = [e[2].elapsed_time(e[3]) for e in evs]
-    ms_step = total_ms / args.steps
-    if pg:
-        t = torch.tensor([ms_step], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms_step = float(t.item())
+    ms_step = max_over_ranks(pg, total_ms / args.steps, dev)
 
     # ---- end to end through the public API with host buffers
     q_h = inp.q.pin_memory()
@@ -335,11 +356,7 @@ def run_gpu(args):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / n_e2e
-    if pg:
-        t = torch.tensor([e2e_ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(pg, e0.elapsed_time(e1) / n_e2e, dev)
     h2d = q_h.numel() * q_h.element_size() + bt_h.numel() * 4 + sl_h.numel() * 4
     if idx_h is not None:
         h2d += idx_h.numel() * 4
@@ -376,7 +393,7 @@ def run_gpu(args):
             "hbm_frac": achieved_gbs / hbm_peak, "tensor_frac": achieved_tf / tc_peak,
             "roofline_frac": max(t_hbm, t_tc) / (dec_avg * 1e-3),
             "combine_ms": sum(comb_ms) / len(comb_ms), "metadata_ms": sum(meta_ms) / len(meta_ms)}
-    value = world * work["flops"] / (ms_step * 1e-3) / 1e12
+    value = job_tflops(world, work["flops"], ms_step)
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None,
@@ -385,7 +402,7 @@ def run_gpu(args):
             "data": "synthetic", "config": workload_config(inp, work),
             "hbm_gbs": world * work["bytes"] / (ms_step * 1e-3) / 1e9,
             "roofline": roof, "clocks": dict(clocks.summary(), remeasured=remeasured),
-            "e2e": {"value": world * work["flops"] / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "e2e": {"value": job_tflops(world, work["flops"], e2e_ms), "unit": "TFLOP/s",
                     "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": 3 * args.steps}
     if world == 1 and not args.no_cpu_baseline:
