@@ -10,7 +10,9 @@
  * restricted by the causal mask t <= seqlen - s_q + i when `causal` is set,
  * or, for sparse decoding, the token positions listed in `indices[b,i,:]`
  * (entries equal to -1 are ignored). An empty key set gives out = 0 and
- * lse = -inf.
+ * lse = -inf. Optional: a per-head attention sink (one more logit with a
+ * zero value, mla_decode_args.sink). With MLA_KV_NVFP4 the rows are 512
+ * values that are both K and V (d_qk = d_v = 512) and the query is NVFP4 too.
  *
  * Sources (web pages on FlashMLA):
  *   - "Qu'est-ce que FlashMLA ?" (topnet.top), sections "Obtenir les
@@ -43,8 +45,8 @@
  *     than its block-table row, a wait that exceeded its time limit) never
  *     trap: the kernel skips the bad item and ORs a bit into a status word
  *     kept in the workspace; read it with mla_query_device_status().
- *   - Only h_kv == 1 (the MLA latent cache), d_qk == 576, d_v == 512 and a
- *     page size of 64 are implemented.
+ *   - Only h_kv == 1 (the MLA latent cache), d_qk == 576 (512 for NVFP4
+ *     rows), d_v == 512 and a page size of 64 are implemented.
  */
 #ifndef MLA_B200_H_
 #define MLA_B200_H_
