@@ -92,9 +92,10 @@ mla_status_t run_decode(const mla_decode_args* a, const int32_t* indices, int to
   const int mode = a->kv_format == MLA_KV_NVFP4 ? kModeNvfp4
                    : topk > 0                  ? (fp8 ? kModeFp8Sparse : kModeSparse)
                                                : (fp8 ? kModeFp8 : kModeBf16);
-  // Q rows of every unit, and (bf16 paged cache only) the cache as
-  // [pages*64 tokens][576 dims]; boxes of 64 x 64 with 128-B swizzle. The FP8
-  // and sparse modes read the cache with cp.async and need no cache map.
+  // Q rows of every unit (not NVFP4: its query is dequantised by the kernel),
+  // and (bf16 paged cache only) the cache as [pages*64 tokens][576 dims];
+  // boxes of 64 x 64 with 128-B swizzle. The FP8, NVFP4 and sparse modes read
+  // the cache with cp.async and need no cache map.
   CUtensorMap tq, tkv;
   std::memset(&tq, 0, sizeof(tq));
   std::memset(&tkv, 0, sizeof(tkv));

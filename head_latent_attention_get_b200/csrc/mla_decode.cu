@@ -1,8 +1,9 @@
 // MLA decode kernel for sm_100a (tcgen05 + TMEM + TMA).
 //
-// Computes, per work unit (request, or (request, query token) when sparse),
-// softmax(scale * Q K^T) V over the unit's keys, with K = whole 576-dim latent
-// row and V = its first 512 dims ("[flashinfer] ... NVFP4 DeepSeek-V4
+// Computes, per work unit (a block of <= 128 query rows of a request, or
+// (request, query token) when sparse), softmax(scale * Q K^T) V over the
+// unit's keys, with K = whole 576-dim latent row and V = its first 512 dims
+// (NVFP4: a 512-value row that is both) ("[flashinfer] ... NVFP4 DeepSeek-V4
 // decoding", README section: one latent row per token is both K and V;
 // FlashMLA-ETAP summary, core mechanism: S = QK^T, P = softmax(S), O = PV).
 //
@@ -23,12 +24,14 @@
 // the PV product rather than held across the softmax, which keeps the rings
 // deep enough to cover the load latency.
 //
-// Warp roles (256 threads; 512 with the FP8 cache or sparse indices):
+// Warp roles (256 threads for the bf16 paged cache; 512 with the FP8 or NVFP4
+// cache or sparse indices):
 //   0 Q (and, bf16 paged, K slices) via TMA   1 S issuer (+ TMEM alloc)
 //   2 O issuer                                 3 V slots via TMA (bf16 paged)
 //   4-7 softmax + epilogue (row r = 16*(warp-4) + lane, lanes 0-15)
-//   8-11 K gather warps, 12-15 V gather warps (FP8 / sparse): cp.async copies
-//       software-pipelined three slots deep; FP8 codes are converted in place.
+//   8-11 K gather warps, 12-15 V gather warps (FP8 / NVFP4 / sparse): cp.async
+//       copies software-pipelined two slots deep; FP8 and NVFP4 codes are
+//       converted to bf16 in place.
 // Every mbarrier wait is bounded; on timeout the CTA records
 // MLA_DEVICE_STATUS_TIMEOUT, stops issuing work, waits (bounded) for its own
 // copies in flight and exits normally. Every ring has exactly one producer
@@ -99,14 +102,14 @@ __device__ __forceinline__ bool group_sync(Ctrl* c, uint64_t* bar, uint32_t& pha
 }
 
 // ============================================================================ gather groups
-// FP8 and sparse modes: four warps fill the K ring and four the V ring with
+// FP8, NVFP4 and sparse modes: four warps fill the K ring and four the V ring with
 // 16-byte cp.async copies. Warp lw of a group owns a quarter of every slot's
 // rows (K: tile rows 32lw..32lw+31; V: page rows 16lw..16lw+15), lane t the
 // source row of one of them; the copies put 4-16 lanes on each row (row
 // pointers by shuffle), FP8 codes are converted in place with four lanes per
 // row. Each warp issues a slot's copies, commits them as one group and retires
 // the slot it issued kLag slots earlier: wait for that group, convert it
-// (FP8), fence the generic-proxy writes for the tensor core, arrive on the
+// (FP8, NVFP4), fence the generic-proxy writes for the tensor core, arrive on the
 // slot's full barrier (count 32 x 4 warps).
 constexpr int kGatherWarps = 4;
 constexpr int kGatherThreads = 32 * kGatherWarps;

@@ -1,6 +1,6 @@
-// MLA decode for units with more than 64 query rows (e.g. 128 heads) on the
-// BF16 cache, paged or token-sparse: one CTA pair (cluster of 2 CTAs on two
-// SMs) per scheduler part.
+// MLA decode for units of 65-128 query rows (e.g. 128 heads, or a 128-row
+// block of a request with more rows) on the BF16 cache, paged or
+// token-sparse: one CTA pair (cluster of 2 CTAs on two SMs) per scheduler part.
 //
 // Same computation as mla_decode.cu -- per unit, softmax(scale * Q K^T) V with
 // K = the 576-dim latent row and V = its first 512 dims ([flashinfer] ...
