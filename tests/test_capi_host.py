@@ -193,3 +193,14 @@ def test_args_struct_layout_matches_header(tmp_path):
     got = [int(x) for x in subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()]
     assert got[0] == ctypes.sizeof(C.MlaDecodeArgs)
     assert got[1:] == [getattr(C.MlaDecodeArgs, f).offset for f in fields]
+
+
+def test_decode_geometry_is_the_fewest_equal_blocks():
+    """For every s_q <= 8 and h_q <= 300: blocks tile the request's rows
+    exactly, hold at most 128 rows, and no smaller block count would do."""
+    for s_q in range(1, 9):
+        for h_q in range(1, 301, 7):
+            upr, rows = M.mla_decode_geometry(s_q, h_q, 1, 0)
+            R = s_q * h_q
+            assert upr * rows == R and rows <= 128
+            assert all(R % n or R // n > 128 for n in range(1, upr))

@@ -69,3 +69,21 @@ def test_algorithmic_work_dsv3_formula():
     a = W.make_inputs(w)
     work = W.algorithmic_work(a)
     assert work["flops"] == 2.0 * (70 + 129) * 16 * (576 + 512)
+
+
+def test_nvfp4_encoder_round_trips_within_half_a_step():
+    """The seeded NVFP4 encoder (data preparation) picks, per value, an E2M1
+    code whose decoded value is within half an E2M1 step of x/scale (times the
+    block scale), and the block maximum maps to 4..6 before saturation."""
+    rng = np.random.default_rng(5)
+    x = torch.from_numpy(rng.standard_normal((64, 512)).astype(np.float32))
+    packed, scales = W.quantize_nvfp4(x)
+    assert packed.shape == (64, 256) and scales.shape == (64, 32) and packed.dtype == torch.uint8
+    dec = O.dequant_nvfp4(packed.numpy(), scales.numpy())
+    sc = np.repeat(O.ue4m3_to_f64(scales.numpy()), 16, axis=-1)
+    y = x.double().numpy() / sc
+    # E2M1 magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6: the gap to a neighbour is at most 2
+    assert np.all(np.abs(dec / sc - np.clip(y, -6, 6)) <= 1.0 + 1e-12)
+    blk_max = np.abs(dec).reshape(64, 32, 16).max(-1) / O.ue4m3_to_f64(scales.numpy())
+    assert np.all((blk_max >= 4.0) | (blk_max == 0)) and np.all(blk_max <= 6.0)
+    assert np.all(scales.numpy() < 0x7F)                               # finite, unsigned scales
