@@ -204,3 +204,20 @@ def test_decode_geometry_is_the_fewest_equal_blocks():
             R = s_q * h_q
             assert upr * rows == R and rows <= 128
             assert all(R % n or R // n > 128 for n in range(1, upr))
+
+
+def test_host_scheduler_random_shapes_with_row_blocks():
+    """Random batches, query tokens, heads (1..300, so up to 18 row-block
+    units per request), sparse or paged, and part counts: every schedule is
+    an exact cover with consistent split counts and balanced parts."""
+    rng = np.random.default_rng(11)
+    for _ in range(60):
+        B = int(rng.integers(1, 40))
+        s_q = int(rng.integers(1, 9))
+        h_q = int(rng.integers(1, 301))
+        sparse = bool(rng.random() < 0.3) and h_q <= 128
+        topk = 64 * int(rng.integers(1, 6)) if sparse else 0
+        lens = rng.integers(0, 9000, size=B)
+        parts = int(rng.integers(1, 160))
+        md, ns = host_schedule(lens, B, s_q, h_q, topk, parts)
+        S.check_schedule(md, ns, lens, B, s_q, topk, parts, h_q=h_q)
