@@ -321,3 +321,121 @@ def reference_decode(inp, requests=None):
                              inp.indices.numpy(), w.scale, requests=requests, sink=sink)
     return decode_dense(q, cache, inp.block_table.numpy(), inp.cache_seqlens.numpy(),
                         w.scale, w.causal, requests=requests, sink=sink)
+
+
+# --------------------------------------------------------------------------
+# the steps around the attention: query norm + RoPE, output conjugate RoPE +
+# FP8 cast ("deepseek-ai/FlashMLA" (agentlenshq), feature list: a fused kernel
+# runs Q-norm, RoPE, the attention, the output-side conjugate RoPE and the
+# final FP8 cast in one launch). The page gives the order of the steps only;
+# the readings below are the plainest ones and are shared with the design doc:
+#   * Q-norm = RMS normalisation of each query row (one head of one query
+#     token) over all of its d_qk values, times a per-dimension weight gamma:
+#     q / sqrt(mean(q^2) + eps) * gamma.
+#   * RoPE acts on the last 64 dims of a row (the RoPE part of the 576-dim
+#     latent row, or of a 512-dim NVFP4 row) and rotates consecutive pairs
+#     (x[2i], x[2i+1]) by the angle theta_i of the query token's position:
+#     (x0 cos - x1 sin, x0 sin + x1 cos). The caller gives cos/sin per query
+#     token and pair, [B, s_q, 32].
+#   * The output's RoPE part is the part of V that lies in those dims: none
+#     for 576-dim rows (V = dims 0..511), dims 448..511 for 512-dim rows. It
+#     is rotated back by the same angle (the conjugate rotation).
+#   * FP8 cast: per 128-value tile of the 512-dim output row, scale =
+#     amax / 448 (1 if amax = 0) and code = e4m3 round-to-nearest-even of
+#     value / scale, saturated to +-448. These integer decisions are taken
+#     in fp32 with every product, sum and quotient rounded once, the
+#     precision of the kernel (the page fixes none).
+# --------------------------------------------------------------------------
+ROPE_DIMS = 64
+E4M3_MAX = 448.0
+
+
+def rms_norm(x, gamma, eps):
+    """x / sqrt(mean(x^2, last axis) + eps) * gamma, in fp64."""
+    x = np.asarray(x, dtype=np.float64)
+    ms = np.mean(x * x, axis=-1, keepdims=True)
+    return x / np.sqrt(ms + float(eps)) * np.asarray(gamma, dtype=np.float64)
+
+
+def rope_rotate(x, cos, sin, conjugate=False):
+    """Rotate consecutive pairs (x[..., 2i], x[..., 2i+1]) by theta_i, given
+    cos/sin [..., n/2] (broadcast against x's leading axes); the conjugate
+    rotation turns by -theta_i. fp64."""
+    x = np.asarray(x, dtype=np.float64)
+    c = np.asarray(cos, dtype=np.float64)
+    s = np.asarray(sin, dtype=np.float64)
+    if conjugate:
+        s = -s
+    x0, x1 = x[..., 0::2], x[..., 1::2]
+    y = np.empty(np.broadcast(x, np.repeat(c, 2, axis=-1)).shape)
+    y[..., 0::2] = x0 * c - x1 * s
+    y[..., 1::2] = x0 * s + x1 * c
+    return y
+
+
+def q_norm_rope(q, gamma, eps, cos, sin):
+    """q [B, s_q, h_q, d] -> RMS-normalised rows (weight gamma [d]) whose last
+    ROPE_DIMS dims are rotated by the query token's angles (cos/sin
+    [B, s_q, 32]). fp64."""
+    y = rms_norm(q, gamma, eps)
+    y[..., -ROPE_DIMS:] = rope_rotate(y[..., -ROPE_DIMS:], np.asarray(cos)[:, :, None, :],
+                                      np.asarray(sin)[:, :, None, :])
+    return y
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """Value (fp64 or fp32) -> OCP E4M3 code: round to the nearest
+    representable value, ties to the even code (mantissa bit 0 clear), with
+    magnitudes beyond 448 saturated to 448; NaN -> 0x7F. The representable
+    magnitudes are m/8 * 2^-6 (m < 8, subnormal) and (1 + m/8) * 2^(e-7)
+    (e = 1..15, excluding e = 15, m = 7)."""
+    x = np.asarray(x, dtype=np.float64)
+    mags = np.array([(m / 8.0) * 2.0 ** -6 for m in range(8)] +
+                    [(1.0 + m / 8.0) * 2.0 ** (e - 7) for e in range(1, 16) for m in range(8)
+                     if not (e == 15 and m == 7)])          # index = code & 0x7F (0..126)
+    a = np.minimum(np.abs(x), E4M3_MAX)
+    hi = np.clip(np.searchsorted(mags, a, side="left"), 0, len(mags) - 1)   # first mag >= a
+    lo = np.maximum(hi - 1, 0)
+    dlo, dhi = a - mags[lo], mags[hi] - a
+    pick_hi = (dhi < dlo) | ((dhi == dlo) & (hi % 2 == 0))
+    code = np.where(pick_hi, hi, lo)
+    code = np.where(a == mags[hi], hi, code).astype(np.int64)
+    code = code | np.where(np.signbit(x), 0x80, 0)
+    code = np.where(np.isnan(x), 0x7F, code)
+    return code.astype(np.uint8)
+
+
+def _f32(v):
+    return np.asarray(v, dtype=np.float32)
+
+
+def fp8_cast_rows(x, tile=128):
+    """fp32 rows [..., n] -> (codes uint8 [..., n], scales fp32 [..., n/tile]).
+    Per tile: amax = max |x|, scale = fp32(amax / 448) (1 if amax = 0),
+    code = e4m3_encode(fp32(x / scale)); each division rounded once in fp32."""
+    x = _f32(x)
+    t = x.reshape(*x.shape[:-1], x.shape[-1] // tile, tile)
+    amax = np.max(np.abs(t), axis=-1)
+    scale = np.where(amax > 0, _f32(amax / np.float32(E4M3_MAX)), np.float32(1.0)).astype(np.float32)
+    q = _f32(t / scale[..., None])
+    return e4m3_encode(q).reshape(x.shape), scale
+
+
+def out_rope_fp8(out, cos, sin, d_qk):
+    """Output epilogue on [B, s_q, h_q, 512] output values (the bf16 results,
+    exact in fp32): the output's RoPE part (dims d_qk-64..d_qk-1 that lie
+    below 512: none for d_qk = 576, 448..511 for d_qk = 512) rotated back by
+    the query token's angle, in fp32 with every product and sum rounded once
+    ((x0 c + x1 s, x1 c - x0 s)), then fp8_cast_rows. Returns (codes, scales,
+    rotated fp32 values)."""
+    y = _f32(out).copy()
+    lo = d_qk - ROPE_DIMS
+    if lo < y.shape[-1]:
+        c = _f32(cos)[:, :, None, :]
+        s = _f32(sin)[:, :, None, :]
+        x0 = y[..., lo::2].copy()
+        x1 = y[..., lo + 1::2].copy()
+        y[..., lo::2] = _f32(_f32(x0 * c) + _f32(x1 * s))
+        y[..., lo + 1::2] = _f32(_f32(x1 * c) - _f32(x0 * s))
+    codes, scales = fp8_cast_rows(y)
+    return codes, scales, y

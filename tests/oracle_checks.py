@@ -514,3 +514,147 @@ def check_nvfp4_decode_brute_force(reference_decode):
             eo, el = _mp_attend(qs, rows[:n], 512 ** -0.5, 512)
             _close(out[b, i], eo, 1e-13)
             _close(lse[b, i], el, 1e-13)
+
+
+# ---------------------------------------------------------------- query norm, RoPE, output FP8 cast
+def check_rms_norm(rms_norm, seeds=range(3)):
+    """Invariants of RMS normalisation: with gamma = 1 and eps = 0 every row
+    has mean square exactly 1; the result does not change when a row is
+    scaled; gamma multiplies per dimension; eps enters under the root, so the
+    mean square becomes ms / (ms + eps)."""
+    for sd in seeds:
+        rng = np.random.default_rng(400 + sd)
+        x = rng.standard_normal((5, 576)) * rng.uniform(0.1, 10, size=(5, 1))
+        one = np.ones(576)
+        y = rms_norm(x, one, 0.0)
+        _close(np.mean(y * y, axis=1), np.ones(5), 1e-12)
+        _close(rms_norm(3.5 * x, one, 0.0), y, 1e-12)
+        g = rng.uniform(-2, 2, size=576)
+        _close(rms_norm(x, g, 0.0), y * g, 1e-12)
+        ms = np.mean(x * x, axis=1)
+        eps = 0.37
+        ye = rms_norm(x, one, eps)
+        _close(np.mean(ye * ye, axis=1), ms / (ms + eps), 1e-12)
+
+
+def check_rope(rope_rotate):
+    """Rotation of consecutive pairs: angle 0 is the identity; a quarter turn
+    maps (x0, x1) to (-x1, x0) with the pairs (2i, 2i+1) (so e_0 goes to e_1,
+    not to e_32); every pair keeps its length; turning by a then b equals
+    turning by a + b; the conjugate undoes the rotation."""
+    rng = np.random.default_rng(410)
+    x = rng.standard_normal((3, 64))
+    z = np.zeros((3, 32))
+    _close(rope_rotate(x, np.ones((3, 32)), z), x, 0)
+    e0 = np.zeros(64)
+    e0[0] = 1.0
+    q = rope_rotate(e0, np.zeros(32), np.ones(32))
+    want = np.zeros(64)
+    want[1] = 1.0
+    _close(q, want, 0)
+    y = rope_rotate(x, np.zeros((3, 32)), np.ones((3, 32)))
+    _close(y[:, 0::2], -x[:, 1::2], 0)
+    _close(y[:, 1::2], x[:, 0::2], 0)
+    a = rng.uniform(-7, 7, size=(3, 32))
+    b = rng.uniform(-7, 7, size=(3, 32))
+    ra = rope_rotate(x, np.cos(a), np.sin(a))
+    _close(np.hypot(ra[:, 0::2], ra[:, 1::2]), np.hypot(x[:, 0::2], x[:, 1::2]), 1e-12)
+    rab = rope_rotate(ra, np.cos(b), np.sin(b))
+    _close(rab, rope_rotate(x, np.cos(a + b), np.sin(a + b)), 1e-12)
+    _close(rope_rotate(ra, np.cos(a), np.sin(a), conjugate=True), x, 1e-12)
+
+
+def check_q_norm_rope(q_norm_rope, rms_norm, rope_rotate):
+    """Only the last 64 dims are rotated, each query token by its own angles
+    (pinned through the two checks above and a per-token comparison)."""
+    rng = np.random.default_rng(420)
+    B, s_q, h, d = 2, 3, 4, 576
+    q = rng.standard_normal((B, s_q, h, d))
+    g = rng.uniform(0.5, 1.5, size=d)
+    th = rng.uniform(-3, 3, size=(B, s_q, 32))
+    y = q_norm_rope(q, g, 1e-6, np.cos(th), np.sin(th))
+    n = rms_norm(q, g, 1e-6)
+    _close(y[..., :d - 64], n[..., :d - 64], 0)
+    for b in range(B):
+        for i in range(s_q):
+            for hh in range(h):
+                r = rope_rotate(n[b, i, hh, d - 64:], np.cos(th[b, i]), np.sin(th[b, i]))
+                _close(y[b, i, hh, d - 64:], r, 1e-12)
+    # a zero angle leaves the normalised row unchanged
+    y0 = q_norm_rope(q, g, 1e-6, np.ones((B, s_q, 32)), np.zeros((B, s_q, 32)))
+    _close(y0, n, 0)
+
+
+def check_e4m3_encode(e4m3_encode, e4m3_to_f64):
+    """Every finite code decodes and re-encodes to itself; the midpoint of
+    two neighbouring codes goes to the one with an even mantissa; values
+    beyond 448 saturate; random in-range values match torch's float8_e4m3fn
+    cast (round to nearest even)."""
+    codes = np.arange(256)
+    vals = e4m3_to_f64(codes)
+    fin = ~np.isnan(vals)
+    assert np.array_equal(e4m3_encode(vals[fin]), codes[fin].astype(np.uint8))
+    pos = [c for c in range(0x7F) if c != 0x7F]
+    for c in pos[:-1]:
+        mid = 0.5 * (vals[c] + vals[c + 1])
+        got = int(e4m3_encode(np.array([mid]))[0])
+        assert got == (c if c % 2 == 0 else c + 1), (c, got)
+        assert int(e4m3_encode(np.array([-mid]))[0]) == (got | 0x80)
+    assert int(e4m3_encode(np.array([1e9]))[0]) == 0x7E
+    assert int(e4m3_encode(np.array([-500.0]))[0]) == 0xFE
+    x = np.random.default_rng(430).standard_normal(50000).astype(np.float32) * 60
+    x = x[np.abs(x) < 448]
+    t = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(e4m3_encode(x), t)
+
+
+def check_fp8_cast_rows(fp8_cast_rows, e4m3_to_f64):
+    """Per 128-value tile: the largest magnitude maps to +-448 exactly (code
+    0x7E / 0xFE), the scale is amax/448, every dequantised value is within
+    half an e4m3 step (2^-4 relative, or 2^-10 scale in the subnormal range)
+    of the input, and an all-zero tile has scale 1 and zero codes."""
+    rng = np.random.default_rng(440)
+    x = (rng.standard_normal((7, 512)) * rng.uniform(1e-3, 30, size=(7, 1))).astype(np.float32)
+    x[3, 128:256] = 0
+    codes, sc = fp8_cast_rows(x)
+    assert codes.shape == x.shape and sc.shape == (7, 4) and sc.dtype == np.float32
+    assert np.all(sc[3, 1] == 1.0) and np.all(codes[3, 128:256] == 0)
+    t = x.reshape(7, 4, 128)
+    ct = codes.reshape(7, 4, 128)
+    deq = e4m3_to_f64(ct) * sc[..., None]
+    for r in range(7):
+        for j in range(4):
+            if r == 3 and j == 1:
+                continue
+            i = int(np.argmax(np.abs(t[r, j])))
+            assert ct[r, j, i] in (0x7E, 0xFE)
+            assert abs(sc[r, j] - np.max(np.abs(t[r, j])) / 448.0) <= 1e-7 * sc[r, j]
+    bound = np.maximum(2.0 ** -4 * np.abs(t), 2.0 ** -10 * sc[..., None]) * (1 + 1e-6)
+    assert np.all(np.abs(deq - t) <= bound)
+
+
+def check_out_rope_fp8(out_rope_fp8, fp8_cast_rows, rope_rotate):
+    """576-dim rows: the output has no RoPE part, so the epilogue is the
+    plain cast. 512-dim rows: dims 448..511 are turned back by the query
+    token's angle (the result matches the fp64 conjugate rotation to fp32
+    rounding) and the other dims are untouched; a rotation then its
+    epilogue returns the original values."""
+    rng = np.random.default_rng(450)
+    B, s_q, h = 2, 2, 3
+    out = rng.standard_normal((B, s_q, h, 512)).astype(np.float32)
+    th = rng.uniform(-3, 3, size=(B, s_q, 32))
+    c, s = np.cos(th).astype(np.float32), np.sin(th).astype(np.float32)
+    codes, sc, y = out_rope_fp8(out, c, s, 576)
+    c2, s2 = fp8_cast_rows(out)
+    assert np.array_equal(codes, c2) and np.array_equal(sc, s2) and np.array_equal(y, out)
+    codes, sc, y = out_rope_fp8(out, c, s, 512)
+    assert np.array_equal(y[..., :448], out[..., :448])
+    ref = rope_rotate(out[..., 448:].astype(np.float64), c[:, :, None, :].astype(np.float64),
+                      s[:, :, None, :].astype(np.float64), conjugate=True)
+    _close(y[..., 448:], ref, 1e-5)
+    rot = rope_rotate(out[..., 448:].astype(np.float64), c[:, :, None, :].astype(np.float64),
+                      s[:, :, None, :].astype(np.float64))
+    full = out.copy()
+    full[..., 448:] = rot.astype(np.float32)
+    _, _, back = out_rope_fp8(full, c, s, 512)
+    _close(back[..., 448:], out[..., 448:], 1e-5)

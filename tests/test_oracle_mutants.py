@@ -247,3 +247,156 @@ def test_nvfp4_layout_mutants_caught(mutant, monkeypatch):
 
 def test_e2m1_bias_mistake_caught():
     assert _fails(C.check_e2m1, _e2m1_bias0)
+
+
+# ---------------------------------------------------------------- query norm, RoPE, output FP8 cast
+def _rms_sum_not_mean(x, gamma, eps):
+    x = np.asarray(x, float)
+    return x / np.sqrt(np.sum(x * x, axis=-1, keepdims=True) + eps) * gamma
+
+
+def _rms_eps_outside(x, gamma, eps):
+    x = np.asarray(x, float)
+    return x / (np.sqrt(np.mean(x * x, axis=-1, keepdims=True)) + eps) * gamma
+
+
+def _rms_no_gamma(x, gamma, eps):
+    return O.rms_norm(x, np.ones(np.shape(x)[-1]), eps)
+
+
+def _rms_no_sqrt(x, gamma, eps):
+    x = np.asarray(x, float)
+    return x / (np.mean(x * x, axis=-1, keepdims=True) + eps) * gamma
+
+
+@pytest.mark.parametrize("mutant", [_rms_sum_not_mean, _rms_eps_outside, _rms_no_gamma, _rms_no_sqrt],
+                         ids=lambda f: f.__name__)
+def test_rms_norm_mutants_caught(mutant):
+    assert _fails(C.check_rms_norm, mutant)
+
+
+def _rope_half_split(x, cos, sin, conjugate=False):
+    x = np.asarray(x, float)
+    n = x.shape[-1] // 2
+    s = -np.asarray(sin) if conjugate else np.asarray(sin)
+    y = np.empty(np.broadcast(x, np.concatenate([cos, cos], axis=-1)).shape)
+    y[..., :n] = x[..., :n] * cos - x[..., n:] * s
+    y[..., n:] = x[..., :n] * s + x[..., n:] * cos
+    return y
+
+
+def _rope_sign_flipped(x, cos, sin, conjugate=False):
+    return O.rope_rotate(x, cos, sin, not conjugate)
+
+
+def _rope_sin_cos_swapped(x, cos, sin, conjugate=False):
+    return O.rope_rotate(x, sin, cos, conjugate)
+
+
+def _rope_conj_ignored(x, cos, sin, conjugate=False):
+    return O.rope_rotate(x, cos, sin, False)
+
+
+@pytest.mark.parametrize("mutant", [_rope_half_split, _rope_sign_flipped, _rope_sin_cos_swapped,
+                                    _rope_conj_ignored], ids=lambda f: f.__name__)
+def test_rope_mutants_caught(mutant):
+    assert _fails(C.check_rope, mutant)
+
+
+def _qnr_rotates_front(q, gamma, eps, cos, sin):
+    y = O.rms_norm(q, gamma, eps)
+    y[..., :64] = O.rope_rotate(y[..., :64], np.asarray(cos)[:, :, None, :], np.asarray(sin)[:, :, None, :])
+    return y
+
+
+def _qnr_rope_before_norm(q, gamma, eps, cos, sin):
+    q = np.array(q, float)
+    q[..., -64:] = O.rope_rotate(q[..., -64:], np.asarray(cos)[:, :, None, :], np.asarray(sin)[:, :, None, :])
+    return O.rms_norm(q, gamma, eps) * 0 + O.q_norm_rope(q, gamma, eps, np.ones_like(cos), np.zeros_like(sin))
+
+
+def _qnr_token0_angles(q, gamma, eps, cos, sin):
+    c = np.repeat(np.asarray(cos)[:, :1], np.shape(cos)[1], axis=1)
+    s = np.repeat(np.asarray(sin)[:, :1], np.shape(sin)[1], axis=1)
+    return O.q_norm_rope(q, gamma, eps, c, s)
+
+
+@pytest.mark.parametrize("mutant", [_qnr_rotates_front, _qnr_rope_before_norm, _qnr_token0_angles],
+                         ids=lambda f: f.__name__)
+def test_q_norm_rope_mutants_caught(mutant):
+    assert _fails(C.check_q_norm_rope, mutant, O.rms_norm, O.rope_rotate)
+
+
+def _enc_truncate(x):
+    """round toward zero instead of to nearest"""
+    x = np.asarray(x, float)
+    v = O.e4m3_to_f64(np.arange(127))
+    a = np.minimum(np.abs(x), 448.0)
+    idx = np.searchsorted(v, a, side="right") - 1
+    return (np.clip(idx, 0, 126) | np.where(np.signbit(x), 0x80, 0)).astype(np.uint8)
+
+
+def _enc_ties_up(x):
+    x = np.asarray(x, float)
+    v = O.e4m3_to_f64(np.arange(127))
+    a = np.minimum(np.abs(x), 448.0)
+    hi = np.clip(np.searchsorted(v, a, side="left"), 0, 126)
+    lo = np.maximum(hi - 1, 0)
+    code = np.where(v[hi] - a <= a - v[lo], hi, lo)
+    return (code | np.where(np.signbit(x), 0x80, 0)).astype(np.uint8)
+
+
+def _enc_no_saturation(x):
+    c = O.e4m3_encode(x)
+    return np.where(np.abs(np.asarray(x, float)) > 448, 0x7F, c).astype(np.uint8)
+
+
+@pytest.mark.parametrize("mutant", [_enc_truncate, _enc_ties_up, _enc_no_saturation], ids=lambda f: f.__name__)
+def test_e4m3_encode_mutants_caught(mutant):
+    assert _fails(C.check_e4m3_encode, mutant, O.e4m3_to_f64)
+
+
+def _cast_scale_fp8max_240(x, tile=128):
+    x = np.asarray(x, np.float32)
+    t = x.reshape(*x.shape[:-1], -1, tile)
+    amax = np.abs(t).max(-1)
+    sc = np.where(amax > 0, amax / np.float32(240.0), 1).astype(np.float32)
+    return O.e4m3_encode((t / sc[..., None]).astype(np.float32)).reshape(x.shape), sc
+
+
+def _cast_tile_64(x, tile=128):
+    return O.fp8_cast_rows(x, 64)
+
+
+def _cast_no_scale(x, tile=128):
+    x = np.asarray(x, np.float32)
+    return O.e4m3_encode(x), np.ones((*x.shape[:-1], x.shape[-1] // tile), np.float32)
+
+
+@pytest.mark.parametrize("mutant", [_cast_scale_fp8max_240, _cast_tile_64, _cast_no_scale],
+                         ids=lambda f: f.__name__)
+def test_fp8_cast_mutants_caught(mutant):
+    assert _fails(C.check_fp8_cast_rows, mutant, O.e4m3_to_f64)
+
+
+def _epi_rotates_forward(out, cos, sin, d_qk):
+    return O.out_rope_fp8(out, cos, -np.asarray(sin), d_qk)
+
+
+def _epi_rotates_576(out, cos, sin, d_qk):
+    return O.out_rope_fp8(out, cos, sin, 512)
+
+
+def _epi_wrong_dims(out, cos, sin, d_qk):
+    y = np.array(out, np.float32)
+    if d_qk == 512:
+        r = O.rope_rotate(y[..., :64], np.asarray(cos)[:, :, None, :], np.asarray(sin)[:, :, None, :], True)
+        y[..., :64] = r.astype(np.float32)
+    c, s = O.fp8_cast_rows(y)
+    return c, s, y
+
+
+@pytest.mark.parametrize("mutant", [_epi_rotates_forward, _epi_rotates_576, _epi_wrong_dims],
+                         ids=lambda f: f.__name__)
+def test_out_epilogue_mutants_caught(mutant):
+    assert _fails(C.check_out_rope_fp8, mutant, O.fp8_cast_rows, O.rope_rotate)

@@ -96,3 +96,27 @@ def test_nvfp4_products_exact_in_bf16():
 
 def test_nvfp4_decode_brute_force():
     C.check_nvfp4_decode_brute_force(O.reference_decode)
+
+
+def test_rms_norm_invariants():
+    C.check_rms_norm(O.rms_norm)
+
+
+def test_rope_pairs():
+    C.check_rope(O.rope_rotate)
+
+
+def test_q_norm_rope():
+    C.check_q_norm_rope(O.q_norm_rope, O.rms_norm, O.rope_rotate)
+
+
+def test_e4m3_encode():
+    C.check_e4m3_encode(O.e4m3_encode, O.e4m3_to_f64)
+
+
+def test_fp8_cast_rows():
+    C.check_fp8_cast_rows(O.fp8_cast_rows, O.e4m3_to_f64)
+
+
+def test_out_rope_fp8():
+    C.check_out_rope_fp8(O.out_rope_fp8, O.fp8_cast_rows, O.rope_rotate)
