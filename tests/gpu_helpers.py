@@ -117,4 +117,14 @@ def oracle_for(inp, requests=None):
     return O.reference_decode(inp, requests=requests)
 
 
+def compare_full(inp, out_gpu, lse_gpu, where, few_keys=False):
+    """Every output row of the batch against the oracle (no sampling): the
+    oracle runs on all requests, the comparison is element by element with
+    the tolerances above (with few_keys, rows of fewer than FEW_KEYS keys get
+    the bf16 bound)."""
+    ref_o, ref_l = O.reference_decode(inp)
+    assert not np.isnan(ref_l).any() and not np.isnan(ref_o).any(), "oracle left rows unset"
+    return compare(out_gpu, lse_gpu, ref_o, ref_l, where, inp=inp if few_keys else None)
+
+
 from workloads.mla_workloads import restrict  # noqa: E402,F401

@@ -66,14 +66,10 @@ def test_row_blocks_fp8(s_q, h_q):
     _check(inp, f"fp8 s_q={s_q} h_q={h_q}")
 
 
-def test_row_blocks_larger_batch_sampled():
-    """64 requests x 6 query tokens x 64 heads, 4096 tokens each; sampled
-    requests checked against the oracle."""
+def test_row_blocks_larger_batch_every_request():
+    """64 requests x 6 query tokens x 64 heads, 4096 tokens each; every
+    request checked against the oracle."""
     w = _dense(batch=64, seqlens=[4096] * 64, s_q=6, h_q=64, causal=True, seed=31)
     inp = W.make_inputs(w)
     out, lse, _ = G.run_gpu(inp)
-    req = [0, 33, 63]
-    sub = G.restrict(inp, req)
-    ref_o, ref_l = G.oracle_for(sub)
-    G.compare(out[req], lse[req], ref_o, ref_l, "s_q=6 h_q=64 sampled")
-    assert np.isfinite(lse).all() and np.isfinite(out).all()
+    G.compare_full(inp, out, lse, "s_q=6 h_q=64", few_keys=True)
