@@ -23,7 +23,6 @@ import json
 import os
 import statistics
 import sys
-import threading
 import time
 
 import numpy as np
@@ -81,56 +80,74 @@ def recorded_traffic(workload: str):
 
 
 class ClockSampler:
-    """Samples SM clock and throttle reasons through NVML while running."""
+    """Samples SM clock and throttle reasons while the timed loop runs.
+
+    A separate `nvidia-smi -lms` process does the sampling, so the Python
+    thread that enqueues the kernels cannot starve it; only samples whose
+    timestamps fall inside the timed window are kept. Falls back to an NVML
+    thread when nvidia-smi is not available."""
 
     REASONS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
                "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
 
-    def __init__(self, device, period_s: float = 0.002):
+    def __init__(self, device, period_ms: int = 20):
         self.samples, self.reasons = [], set()
-        self.period = period_s
-        self.stop_evt = threading.Event()
-        self.ok = False
+        self.period_ms = period_ms
         self.max_mhz = None
+        self.proc = None
+        self.source = None
         try:
-            import pynvml
-            pynvml.nvmlInit()
-            self.nv = pynvml
-            uuid = str(torch.cuda.get_device_properties(device).uuid)
-            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
-            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
-            self.ok = True
+            self.uuid = str(torch.cuda.get_device_properties(device).uuid)
+            if not self.uuid.startswith("GPU-"):
+                self.uuid = "GPU-" + self.uuid
         except Exception:
-            self.ok = False
-
-    def _run(self):
-        while not self.stop_evt.is_set():
-            try:
-                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
-                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                for name, bit in self.REASONS.items():
-                    if r & bit:
-                        self.reasons.add(name)
-            except Exception:
-                pass
-            time.sleep(self.period)
+            self.uuid = None
 
     def __enter__(self):
-        if self.ok:
-            self.t = threading.Thread(target=self._run, daemon=True)
-            self.t.start()
+        import subprocess
+        if self.uuid:
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", "-i", self.uuid, "--query-gpu=timestamp,clocks.sm,clocks.max.sm,"
+                     "clocks_event_reasons.active", "--format=csv,noheader,nounits", "-lms", str(self.period_ms)],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                self.proc.stdout.readline()   # sampling has started
+                self.source = "nvidia-smi"
+            except Exception:
+                self.proc = None
+        self.t0 = time.time()
         return self
 
     def __exit__(self, *a):
-        if self.ok:
-            self.stop_evt.set()
-            self.t.join()
+        self.t1 = time.time()
+        if self.proc is None:
+            return
+        import datetime
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        for line in out.splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 4:
+                continue
+            try:
+                ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                mhz, mx, bits = float(f[1]), float(f[2]), int(f[3], 16)
+            except ValueError:
+                continue
+            if self.t0 - 0.05 <= ts <= self.t1 + 0.05:
+                self.samples.append(mhz)
+                self.max_mhz = mx
+                for name, bit in self.REASONS.items():
+                    if bits & bit:
+                        self.reasons.add(name)
 
     def summary(self):
-        if not self.ok or not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["nvml unavailable"]}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["no clock samples"],
+                    "samples": 0}
         return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+                "reasons": sorted(self.reasons), "samples": len(self.samples), "source": self.source,
+                "window_s": round(self.t1 - self.t0, 3)}
 
 
 def workload_config(inp, work):
@@ -140,8 +157,10 @@ def workload_config(inp, work):
            "causal": w.causal, "softmax_scale": w.scale,
            "tokens_cached": int(sum(int(x) for x in inp.cache_seqlens.tolist())),
            "algorithmic_flops": work["flops"], "algorithmic_bytes": work["bytes"],
-           "l2": "inputs larger than L2 (cache %.0f MB > 126 MB), no flush" % (
-               inp.kcache.numel() * inp.kcache.element_size() / 1e6)}
+           "l2": ("a step reads %.0f MB (more than twice the 126 MB L2), no flush" if
+                  work["bytes"] >= 2 * L2_BYTES else
+                  "a step reads %.0f MB (less than twice L2): 256 MB written before every step") % (
+               work["bytes"] / 1e6)}
     if w.topk:
         cfg["topk"] = w.topk
     if inp.sink is not None:
@@ -170,7 +189,8 @@ def oracle_sample(inp, budget_s: float):
         if elapsed >= budget_s:
             break
     threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    return {"value": flops / elapsed / 1e12, "unit": "TFLOP/s", "cores": int(threads), "kind": "oracle",
+    return {"value": flops / elapsed / 1e12, "unit": "TFLOP/s", "cores": int(threads),
+            "host_cores": os.cpu_count(), "kind": "oracle",
             "sample": f"{len(done)} of {w.batch} requests of the workload (whole requests, "
                       f"{flops:.3g} FLOPs in {elapsed:.2f} s)"}
 
@@ -202,7 +222,8 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / len(times),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": workload_config(inp, work),
-            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": int(threads), "kind": "oracle",
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": int(threads),
+                             "host_cores": os.cpu_count(), "kind": "oracle",
                              "sample": "one whole request of the workload per step"},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -242,37 +263,45 @@ def job_tflops(world: int, flops_per_rank: float, ms: float) -> float:
 
 
 # ----------------------------------------------------------------------------- GPU path
-def run_gpu(args):
+L2_BYTES = 126 * 2 ** 20
+CONFIGS = ["tiny", "dsv3", "mtp", "fp8", "sparse"]   # the five configurations, in order
+
+
+def build_runner(inp, dev, M, C):
+    w = inp.workload
+    d = {k: (None if v is None else v.to(dev)) for k, v in dict(
+        q=inp.q, kc=inp.kcache, bt=inp.block_table, sl=inp.cache_seqlens, idx=inp.indices, sink=inp.sink,
+        qs=inp.q_scale, ks=inp.kv_scale).items()}
+    runner = M.DecodeRunner(d["q"], d["kc"], d["bt"], d["sl"], softmax_scale=w.scale, causal=w.causal,
+                            indices=d["idx"], sink=d["sink"], q_scale=d["qs"], kv_scale=d["ks"])
+    return runner, d
+
+
+def measure(inp, steps: int, warmup: int, dev, pg=None):
+    """Times `steps` decode steps (scheduler + decode kernel + combine) on
+    resident inputs with CUDA events on the launching stream: once back to
+    back (the step time), then again with an event around each kernel (the
+    per-kernel times). The decode kernel is launched with the combine held
+    back and the combine enqueued right after it, so each kernel has its own
+    events. When the bytes a step reads are less than twice L2 (the tiny and
+    token-sparse workloads), a 256 MB buffer is written before each step
+    (outside the per-kernel events) so that every step reads from HBM."""
     import head_latent_attention_get_b200 as M
     from head_latent_attention_get_b200 import _capi as C
-
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    world, rank, local, pg = init_ranks(dev, "nccl")
-
-    inp = W.make_inputs(W.get_workload(args.workload))
-    if args.sink:
-        inp = W.with_sink(inp, seed=inp.workload.seed)
-    work = W.algorithmic_work(inp)
     w = inp.workload
-    q = inp.q.to(dev)
-    kc = inp.kcache.to(dev)
-    bt = inp.block_table.to(dev)
-    sl = inp.cache_seqlens.to(dev)
-    idx = inp.indices.to(dev) if inp.indices is not None else None
-    sink = inp.sink.to(dev) if inp.sink is not None else None
-    qs = inp.q_scale.to(dev) if inp.q_scale is not None else None
-    ks = inp.kv_scale.to(dev) if inp.kv_scale is not None else None
-    runner = M.DecodeRunner(q, kc, bt, sl, softmax_scale=w.scale, causal=w.causal, indices=idx, sink=sink,
-                            q_scale=qs, kv_scale=ks)
-    # timing variant: the decode kernel alone, then the combine enqueued by the caller
+    runner, d = build_runner(inp, dev, M, C)
     runner.args.debug_flags = C.MLA_DEBUG_SKIP_COMBINE
     U, R, P = runner.units, runner.rows, runner.parts
     ws_bytes = runner.workspace.numel()
     stream = torch.cuda.current_stream()
+    # the bytes a step touches (not the whole cache: a token-sparse step reads
+    # only its indexed rows) decide whether L2 could serve the next step
+    touched = W.algorithmic_work(inp)["bytes"]
+    flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev) if touched < 2 * L2_BYTES else None
 
     def step(ev=None):
+        if flush is not None:
+            flush.fill_(1)
         if ev is not None:
             ev[0].record(stream)
         runner.plan(stream)
@@ -281,19 +310,18 @@ def run_gpu(args):
         runner.run(stream)
         if ev is not None:
             ev[2].record(stream)
-        M.mla_combine_sink(runner.workspace, ws_bytes, runner.num_splits, U, R, P, w.h_q, sink, runner.out,
+        M.mla_combine_sink(runner.workspace, ws_bytes, runner.num_splits, U, R, P, w.h_q, d["sink"], runner.out,
                            runner.lse, stream)
         if ev is not None:
             ev[3].record(stream)
 
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         step()
     torch.cuda.synchronize()
     code, bits = runner.status()
     if code != C.MLA_OK:
-        raise RuntimeError(f"device status after warm-up: {M.mla_status_string(code)} bits={bits}")
-
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+        raise RuntimeError(f"{w.name}: device status after warm-up: {M.mla_status_string(code)} bits={bits}")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     bad_reasons = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
@@ -303,10 +331,14 @@ def run_gpu(args):
             pg.barrier()
         torch.cuda.synchronize()
         with ClockSampler(dev) as clocks:
+            # whole steps back to back (the kernels of a step overlap their
+            # launches), then the same steps with an event around each kernel
             t_start.record(stream)
-            for s in range(args.steps):
-                step(evs[s])
+            for s in range(steps):
+                step()
             t_end.record(stream)
+            for s in range(steps):
+                step(evs[s])
             torch.cuda.synchronize()
         if pg:
             pg.barrier()
@@ -314,11 +346,63 @@ def run_gpu(args):
             remeasured = True      # slowdown seen while timing: measure once more
             continue
         break
-    total_ms = t_start.elapsed_time(t_end)
-    meta_ms = [e[0].elapsed_time(e[1]) for e in evs]
-    dec_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    comb_ms = [e[2].elapsed_time(e[3]) for e in evs]
-    ms_step = max_over_ranks(pg, total_ms / args.steps, dev)
+    meta = [e[0].elapsed_time(e[1]) for e in evs]
+    dec = [e[1].elapsed_time(e[2]) for e in evs]
+    comb = [e[2].elapsed_time(e[3]) for e in evs]
+    return {"runner": runner, "rows": runner.rows, "dev_inputs": d, "total_ms": t_start.elapsed_time(t_end), "steps": steps,
+            "flushed": flush is not None, "metadata_ms": sum(meta) / steps, "kernel_ms": sum(dec) / steps,
+            "combine_ms": sum(comb) / steps, "step_kernels_ms": (sum(meta) + sum(dec) + sum(comb)) / steps,
+            "clocks": dict(clocks.summary(), remeasured=remeasured), "launches": 3 * steps}
+
+
+def roofline_of(inp, m, peaks, peak_src):
+    """Roofline figures of the decode kernel from its measured average time."""
+    w = inp.workload
+    work = W.algorithmic_work(inp)
+    hbm_peak = float(peaks["hbm_gbs"])
+    tc_peak = float(peaks["bf16_tflops"])
+    k_ms = m["kernel_ms"]
+    achieved_gbs = work["bytes"] / (k_ms * 1e-3) / 1e9
+    achieved_tf = work["flops"] / (k_ms * 1e-3) / 1e12
+    t_hbm = work["bytes"] / (hbm_peak * 1e9)
+    t_tc = work["flops"] / (tc_peak * 1e12)
+    bound = "hbm" if t_hbm >= t_tc else "tensor"
+    mhz = m["clocks"].get("sm_mhz")
+    return {"bound": bound,
+            "achieved": achieved_gbs if bound == "hbm" else achieved_tf,
+            "peak": hbm_peak if bound == "hbm" else tc_peak,
+            "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
+            "frac": (achieved_gbs / hbm_peak) if bound == "hbm" else (achieved_tf / tc_peak),
+            "traffic": recorded_traffic(w.name),
+            "peak_source": f"{peak_src} (MEASURED_PEAKS.json burst figures)" if peak_src == "measured"
+            else "fallback",
+            "kernel": decode_kernel_name(w, m["rows"]),
+            "kernel_ms": k_ms,
+            "kernel_kclk_at_median_sm_mhz": None if mhz is None else k_ms * mhz,
+            "achieved_tflops": achieved_tf, "achieved_gbs": achieved_gbs,
+            "hbm_frac": achieved_gbs / hbm_peak, "tensor_frac": achieved_tf / tc_peak,
+            "roofline_frac": max(t_hbm, t_tc) / (k_ms * 1e-3),
+            "combine_ms": m["combine_ms"], "metadata_ms": m["metadata_ms"]}
+
+
+def run_gpu(args):
+    import head_latent_attention_get_b200 as M
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    world, rank, local, pg = init_ranks(dev, "nccl")
+    peaks, peak_src = load_peaks()
+
+    inp = W.make_inputs(W.get_workload(args.workload))
+    if args.sink:
+        inp = W.with_sink(inp, seed=inp.workload.seed)
+    work = W.algorithmic_work(inp)
+    w = inp.workload
+    m = measure(inp, args.steps, args.warmup, dev, pg)
+    ms_step = max_over_ranks(pg, m["total_ms"] / args.steps, dev)
+    runner, d = m["runner"], m["dev_inputs"]
+    stream = torch.cuda.current_stream()
 
     # ---- end to end through the public API with host buffers
     q_h = inp.q.pin_memory()
@@ -328,17 +412,17 @@ def run_gpu(args):
     qs_h = inp.q_scale.pin_memory() if inp.q_scale is not None else None
     out_h = torch.empty(runner.out.shape, dtype=runner.out.dtype).pin_memory()
     lse_h = torch.empty(runner.lse.shape, dtype=runner.lse.dtype).pin_memory()
-    runner_e2e = M.DecodeRunner(q, kc, bt, sl, softmax_scale=w.scale, causal=w.causal, indices=idx, sink=sink,
-                                q_scale=qs, kv_scale=ks)
+    runner_e2e = M.DecodeRunner(d["q"], d["kc"], d["bt"], d["sl"], softmax_scale=w.scale, causal=w.causal,
+                                indices=d["idx"], sink=d["sink"], q_scale=d["qs"], kv_scale=d["ks"])
 
     def e2e_step():
-        q.copy_(q_h, non_blocking=True)
-        bt.copy_(bt_h, non_blocking=True)
-        sl.copy_(sl_h, non_blocking=True)
-        if idx is not None:
-            idx.copy_(idx_h, non_blocking=True)
-        if qs is not None:
-            qs.copy_(qs_h, non_blocking=True)
+        d["q"].copy_(q_h, non_blocking=True)
+        d["bt"].copy_(bt_h, non_blocking=True)
+        d["sl"].copy_(sl_h, non_blocking=True)
+        if idx_h is not None:
+            d["idx"].copy_(idx_h, non_blocking=True)
+        if qs_h is not None:
+            d["qs"].copy_(qs_h, non_blocking=True)
         runner_e2e.plan(stream)
         runner_e2e.run(stream)
         out_h.copy_(runner_e2e.out, non_blocking=True)
@@ -362,6 +446,25 @@ def run_gpu(args):
     if qs_h is not None:
         h2d += qs_h.numel()
     d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * 4
+    del runner_e2e
+
+    # ---- the other configurations, timed the same way in the same run (rank 0 reports them)
+    per_config = {}
+    if not args.no_per_config:
+        for name in CONFIGS:
+            if name == args.workload and not args.sink:
+                continue
+            pi = W.make_inputs(W.get_workload(name))
+            pm = measure(pi, min(args.steps, args.per_config_steps), args.warmup, dev, pg)
+            r = roofline_of(pi, pm, peaks, peak_src)
+            r.update({"workload": W.get_workload(name).note, "steps": pm["steps"],
+                      "l2_flush_between_steps": pm["flushed"], "clocks": pm["clocks"],
+                      # with an L2 flush in every step, the step time is the sum of its kernels
+                      "step_ms": pm["step_kernels_ms"] if pm["flushed"] else pm["total_ms"] / pm["steps"]})
+            r["step_tflops"] = W.algorithmic_work(pi)["flops"] / (r["step_ms"] * 1e-3) / 1e12
+            per_config[name] = r
+            del pm
+            torch.cuda.empty_cache()
 
     if pg:
         pg.barrier()
@@ -369,29 +472,7 @@ def run_gpu(args):
     if rank != 0:
         return 0
 
-    peaks, peak_src = load_peaks()
-    hbm_peak = float(peaks["hbm_gbs"])
-    tc_peak = float(peaks["bf16_tflops"])
-    dec_avg = sum(dec_ms) / len(dec_ms)
-    achieved_gbs = work["bytes"] / (dec_avg * 1e-3) / 1e9
-    achieved_tf = work["flops"] / (dec_avg * 1e-3) / 1e12
-    t_hbm = work["bytes"] / (hbm_peak * 1e9)
-    t_tc = work["flops"] / (tc_peak * 1e12)
-    bound = "hbm" if t_hbm >= t_tc else "tensor"
-    traffic = recorded_traffic(w.name)
-    roof = {"bound": bound,
-            "achieved": achieved_gbs if bound == "hbm" else achieved_tf,
-            "peak": hbm_peak if bound == "hbm" else tc_peak,
-            "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
-            "frac": (achieved_gbs / hbm_peak) if bound == "hbm" else (achieved_tf / tc_peak),
-            "traffic": traffic,
-            "peak_source": f"{peak_src} (MEASURED_PEAKS.json burst figures)" if peak_src == "measured"
-            else "fallback",
-            "kernel": decode_kernel_name(w, runner.rows),
-            "kernel_ms": dec_avg,
-            "hbm_frac": achieved_gbs / hbm_peak, "tensor_frac": achieved_tf / tc_peak,
-            "roofline_frac": max(t_hbm, t_tc) / (dec_avg * 1e-3),
-            "combine_ms": sum(comb_ms) / len(comb_ms), "metadata_ms": sum(meta_ms) / len(meta_ms)}
+    roof = roofline_of(inp, m, peaks, peak_src)
     value = job_tflops(world, work["flops"], ms_step)
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -400,10 +481,12 @@ def run_gpu(args):
                       "nvfp4": "nvfp4 (e2m1 + ue4m3) query and cache, dequantised exactly to bf16 mma"}[w.kv],
             "data": "synthetic", "config": workload_config(inp, work),
             "hbm_gbs": world * work["bytes"] / (ms_step * 1e-3) / 1e9,
-            "roofline": roof, "clocks": dict(clocks.summary(), remeasured=remeasured),
+            "roofline": roof, "clocks": m["clocks"],
             "e2e": {"value": job_tflops(world, work["flops"], e2e_ms), "unit": "TFLOP/s",
                     "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": 3 * args.steps}
+            "gpu_launches": m["launches"]}
+    if per_config:
+        line["per_config"] = per_config
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_sample(inp, args.cpu_budget)
     print(json.dumps(line), flush=True)
@@ -421,6 +504,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true", help="time only the chosen workload")
+    ap.add_argument("--per-config-steps", type=int, default=1000,
+                    help="timed steps of each of the other configurations (capped by --steps)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)   # at least 3 untimed warm-up steps
     if args.impl == "reference":

@@ -93,6 +93,11 @@ def lib() -> ctypes.CDLL:
         L.mla_query_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32), vp]
         L.mla_clear_device_status.restype = i
         L.mla_clear_device_status.argtypes = [vp, vp]
+        f = ctypes.c_float
+        L.mla_q_norm_rope.restype = i
+        L.mla_q_norm_rope.argtypes = [vp, vp, i, i, i, i, vp, f, vp, vp, vp]
+        L.mla_out_rope_fp8.restype = i
+        L.mla_out_rope_fp8.argtypes = [vp, i, i, i, i, vp, vp, vp, vp, vp]
         _lib = L
     return _lib
 
@@ -216,3 +221,13 @@ def mla_query_device_status(workspace, stream=None):
 
 def mla_clear_device_status(workspace, stream=None):
     _check(lib().mla_clear_device_status(_ptr(workspace), _stream(stream)), "mla_clear_device_status")
+
+
+def mla_q_norm_rope(q, q_out, batch, s_q, h_q, d_qk, gamma, eps, rope_cos, rope_sin, stream=None):
+    _check(lib().mla_q_norm_rope(_ptr(q), _ptr(q_out), batch, s_q, h_q, d_qk, _ptr(gamma), float(eps),
+                                 _ptr(rope_cos), _ptr(rope_sin), _stream(stream)), "mla_q_norm_rope")
+
+
+def mla_out_rope_fp8(out, batch, s_q, h_q, d_qk, rope_cos, rope_sin, out_fp8, out_scale, stream=None):
+    _check(lib().mla_out_rope_fp8(_ptr(out), batch, s_q, h_q, d_qk, _ptr(rope_cos), _ptr(rope_sin),
+                                  _ptr(out_fp8), _ptr(out_scale), _stream(stream)), "mla_out_rope_fp8")

@@ -109,8 +109,8 @@ __device__ __forceinline__ bool group_sync(Ctrl* c, uint64_t* bar, uint32_t& pha
 // pointers by shuffle), FP8 codes are converted in place with four lanes per
 // row. Each warp issues a slot's copies, commits them as one group and retires
 // the slot it issued kLag slots earlier: wait for that group, convert it
-// (FP8, NVFP4), fence the generic-proxy writes for the tensor core, arrive on the
-// slot's full barrier (count 32 x 4 warps).
+// (FP8, NVFP4), fence the generic-proxy writes for the tensor core, and one
+// lane arrives on the slot's full barrier (count: 4 warps).
 constexpr int kGatherWarps = 4;
 constexpr int kGatherThreads = 32 * kGatherWarps;
 
@@ -232,8 +232,9 @@ __device__ __forceinline__ void retire_slot(const GatherRing& g, int seq, int lw
       }
     }
   }
-  fence_proxy_async_smem();
-  mbar_arrive(&g.full[slot]);
+  fence_proxy_async_smem();  // this lane's rows -> the tensor core
+  __syncwarp();
+  if (t == 0) mbar_arrive(&g.full[slot]);  // one arrival per warp (a per-thread one costs more)
 }
 
 // Source row of tile-relative token tt of tile k (FP8 record, or bf16 cache
@@ -380,7 +381,7 @@ __global__ void __launch_bounds__(MODE == kModeBf16 ? 256 : 256 + 2 * kGatherThr
   const int part = blockIdx.x, rg = blockIdx.y;
   const int row0 = rg * kRowsPerCta;                    // first row of this CTA within a unit
   const int rows_here = min(kRowsPerCta, p.rows - row0);
-  constexpr uint32_t kFullCount = MODE == kModeBf16 ? 1 : kGatherThreads;
+  constexpr uint32_t kFullCount = MODE == kModeBf16 ? 1 : kGatherWarps;  // TMA producer, or one per gather warp
 
   if (threadIdx.x == 0) {
     mbar_init(&c->q_full, 1);
@@ -411,6 +412,7 @@ __global__ void __launch_bounds__(MODE == kModeBf16 ? 256 : 256 + 2 * kGatherThr
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = c->tmem_base;
+  griddep_wait();  // the scheduler's output (and every input) is ready
 
   PieceIter it;
   it.init(p, part);
@@ -803,6 +805,7 @@ __global__ void __launch_bounds__(MODE == kModeBf16 ? 256 : 256 + 2 * kGatherThr
   }
 
   // ---------------------------------------------------------------- teardown
+  griddep_launch_dependents();  // the combine may be scheduled (it waits for this grid)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -817,9 +820,9 @@ static cudaError_t launch_one(const CUtensorMap& tq, const CUtensorMap& tkv, con
   auto kern = mla_decode_kernel<NR, MODE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(parts, row_groups);
-  kern<<<grid, MODE == kModeBf16 ? 256 : 256 + 2 * kGatherThreads, smem, stream>>>(tq, tkv, p);
-  return cudaGetLastError();
+  e = launch_pdl(kern, dim3(parts, row_groups), dim3(MODE == kModeBf16 ? 256 : 256 + 2 * kGatherThreads), smem,
+                 stream, tq, tkv, p);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_decode(int rows_per_cta, int mode, const CUtensorMap& tq, const CUtensorMap& tkv,

@@ -50,13 +50,13 @@
 namespace mla {
 namespace pair {
 
-constexpr int kN = 5;                // ring slots of 16 KB: a K slice (128 tokens x 64 dims)
+constexpr int kN = 7;                // ring slots of 16 KB: a K slice (128 tokens x 64 dims)
                                      // or a V slot (64 tokens x 128 value dims, two 8 KB halves)
 constexpr int kSlot = 16384;
 constexpr int kThreads = 256;         // paged
 constexpr int kThreadsSparse = 320;   // + four cp.async loader warps (2, 3, 8, 9)
 constexpr int kQBytes = 9 * 8192;    // 64 rows x 576 dims
-constexpr int kPBytes = 4 * 8192;    // 64 rows x 256 tokens, per buffer
+constexpr int kPBytes = 4 * 8192;    // 64 rows x 256 tokens (one buffer)
 constexpr int kTmemCols = 512;
 constexpr int kTmemS = 256;          // S buffers at columns 256 and 384; O at 0 and 128
 constexpr float kRescaleLog2 = 8.0f;
@@ -65,7 +65,7 @@ struct Smem {
   static constexpr int q = 0;
   static constexpr int ring = q + kQBytes;
   static constexpr int pt = ring + kN * kSlot;
-  static constexpr int ctrl = pt + 2 * kPBytes;
+  static constexpr int ctrl = pt + kPBytes;
   static constexpr int total = ctrl + 2048;
 };
 
@@ -222,6 +222,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SPARSE ? kThreadsSpa
   cluster_sync_all();  // barriers initialised and TMEM allocated in both CTAs
   tc_fence_after();
   const uint32_t tmem = c->tmem_base;
+  griddep_wait();  // the scheduler's output (and every input) is ready
 
   PieceIter it;
   it.init(p, part);
@@ -436,7 +437,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SPARSE ? kThreadsSpa
         const int nslots = 17 * ((pc.t1 - pc.t0 + 1) >> 1);  // 9 K slices + 8 V slots per step
         for (int i = 0; i < nslots; ++i, ++sc) {
           if (!pwait(pr, &c->v_loc[sc % kN], (sc / kN) & 1, p)) { stop = true; break; }
-          arrive_leader(pr, &c->full[sc % kN]);
+          // relaxed: a release arrive would first wait for this thread's
+          // earlier memory operations (~0.8K clk after cp.async traffic
+          // instead of ~0.1K); the data it signals has landed (v_loc)
+          mbar_arrive_relaxed_cluster(map_to_rank(smem_u32(&c->full[sc % kN]), 0));
         }
       }
     }
@@ -479,7 +483,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SPARSE ? kThreadsSpa
             const bool first = g == 0;
             if (first && pi > 0 && !pwait(pr, &c->o_free, (pi - 1) & 1, p)) { stop = true; break; }
             if (!pwait(pr, &c->p_full[go & 1], (go >> 1) & 1, p)) { stop = true; break; }
-            const uint32_t pt = smem_u32(sP + (go & 1) * kPBytes);
+            const uint32_t pt = smem_u32(sP);
             for (int q = 0; q < 4 && !stop; ++q) {
               for (int jd = 0; jd < 2; ++jd, ++sc) {
                 const int slot = sc % kN;
@@ -563,23 +567,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SPARSE ? kThreadsSpa
           m_used = tmax;
           l_sum *= alpha;
         }
-        // P buffer b was last read by the O product of step gt - 2 (one
-        // barrier per buffer: O of step gt cannot complete before this
-        // thread's P, so the parity wait never falls two phases behind)
-        if (gt >= 2 && !pwait(pr, &c->o_done[b], ((gt >> 1) - 1) & 1, p)) { stop = true; break; }
-        // pass 2: probabilities (masked by select) -> bf16 -> P buffer b,
+        // pass 2: probabilities (masked by select) -> bf16 -> the P buffer,
         // K-major [64 rows][64 keys] per slice: keys 64s.. in slice s; this
-        // thread's keys are 128*half + [0,128), slices 2*half and 2*half + 1
+        // thread's keys are 128*half + [0,128), slices 2*half and 2*half + 1.
+        // The single P buffer was last read by the O product of step gt - 1,
+        // which must also be complete before O is rescaled. (O of step gt + 1,
+        // the next completion of the same barrier, needs this thread's P, so
+        // the parity wait never falls two phases behind.) Half of the
+        // probabilities are computed into registers while that product runs.
         const float mc = (m_used == -INFINITY ? 0.f : m_used) * p.scale_log2;
         float part = 0.f;
-        uint8_t* pbuf = sP + b * kPBytes;
-#pragma unroll 1
-        for (int w = 0; w < 4; ++w) {
+        auto probs = [&](int w, uint32_t (&pk)[16]) {
           uint32_t sv[32];
           tmem_ld32(s_addr + 32 * w, sv);
           tmem_ld_wait();
           const uint32_t mw = pick4u(vm, w);
-          uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const float e0 = ex2_approx(fmaf(__uint_as_float(sv[2 * i]), p.scale_log2, -mc));
@@ -589,19 +591,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SPARSE ? kThreadsSpa
             pk[i] = pack_bf16x2(p0, p1);
             part += p0 + p1;
           }
-          uint8_t* rowp = pbuf + (2 * half + (w >> 1)) * 8192 + (row >> 3) * 1024 + (row & 7) * 128;
+        };
+        auto store = [&](int w, const uint32_t (&pk)[16]) {
+          uint8_t* rowp = sP + (2 * half + (w >> 1)) * 8192 + (row >> 3) * 1024 + (row & 7) * 128;
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const int ch = 4 * (w & 1) + q;
             *reinterpret_cast<uint4*>(rowp + ((ch ^ (row & 7)) << 4)) =
                 make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
           }
+        };
+        {
+          uint32_t pk[2][16];
+#pragma unroll
+          for (int w = 0; w < 2; ++w) probs(w, pk[w]);
+          if (gt >= 1 && !pwait(pr, &c->o_done[(gt - 1) & 1], ((gt - 1) >> 1) & 1, p)) { stop = true; break; }
+#pragma unroll
+          for (int w = 0; w < 2; ++w) store(w, pk[w]);
+#pragma unroll 1
+          for (int w = 2; w < 4; ++w) {
+            probs(w, pk[0]);
+            store(w, pk[0]);
+          }
         }
+        tc_fence_after();
         l_sum += part;
         if (need) {
-          // O must hold every product up to step gt - 1 before it is rescaled
-          if (!pwait(pr, &c->o_done[(gt - 1) & 1], ((gt - 1) >> 1) & 1, p)) { stop = true; break; }
-          tc_fence_after();
+          // O holds every product up to step gt - 1 (waited for above)
 #pragma unroll 1
           for (int c16 = 0; c16 < 16; ++c16) {  // 2 x 128 columns of this row
             uint32_t ov[16];
@@ -672,9 +688,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SPARSE ? kThreadsSpa
   }
 
   // ---------------------------------------------------------------- teardown
-  // Copies this CTA issued whose completion is counted on the other CTA's
-  // barrier cannot be waited for here; after an abort give them time to land.
-  if (aborted(pr)) __nanosleep(100000);
+  // In a normal exit every copy has landed: each slot and Q phase was
+  // consumed by the MMA issuer, and the producer drained its last phases.
+  // After an abort (a bounded wait ran out), a copy this CTA issued may still
+  // be in flight, and when its completion is counted on the other CTA's
+  // barrier no wait here can observe it. Such copies read resident cache
+  // pages and land within microseconds, so the CTA holds its shared memory
+  // for a fixed 200 us of wall time (%globaltimer, not a sleep hint that may
+  // return early) before the final cluster barrier; this bounds the window,
+  // it does not prove every copy landed.
+  if (aborted(pr)) {
+    const uint64_t t0 = global_timer_ns();
+    while (global_timer_ns() - t0 < 200000) {
+    }
+  }
+  griddep_launch_dependents();  // the combine may be scheduled (it waits for this grid)
   tc_fence_before();
   __syncthreads();
   cluster_sync_all();  // no pair MMA, copy or remote arrive of either CTA is still pending
@@ -690,8 +718,8 @@ cudaError_t launch_decode_pair(const CUtensorMap& tq, const CUtensorMap& tkv, co
   auto kern = sparse ? pair::mla_decode_pair_kernel<true> : pair::mla_decode_pair_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  kern<<<2 * parts, sparse ? pair::kThreadsSparse : pair::kThreads, smem, stream>>>(tq, tkv, p);
-  return cudaGetLastError();
+  e = launch_pdl(kern, dim3(2 * parts), dim3(sparse ? pair::kThreadsSparse : pair::kThreads), smem, stream, tq, tkv, p);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 int max_pair_clusters() {

@@ -58,6 +58,26 @@ __device__ __forceinline__ float fold_sink(float& lse, float sigma) {
 }
 #endif
 
+// Launch with programmatic stream serialization: the kernel may start while
+// the previous kernel of the stream finishes (it calls griddep_wait before
+// touching global memory), which hides the launch gap between the scheduler,
+// decode and combine kernels of a step.
+template <typename... Params, typename... Args>
+cudaError_t launch_pdl(void (*kern)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...);
+}
+
 cudaError_t launch_decode(int rows_per_cta, int mode, const CUtensorMap& tq, const CUtensorMap& tkv,
                           const DecodeParams& p, int parts, int row_groups, cudaStream_t stream);
 // Units of more than 64 rows, BF16 cache (paged, or token-sparse when `sparse`):

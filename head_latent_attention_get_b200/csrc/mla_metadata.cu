@@ -21,6 +21,7 @@
 #include <cuda_runtime.h>
 
 #include "mla_kernels.cuh"
+#include "sm100_ptx.cuh"
 
 namespace mla {
 
@@ -153,6 +154,7 @@ __global__ void __launch_bounds__(kMetaThreads) mla_metadata_kernel(const int32_
                                                                    int U, int upr, int topk, int parts,
                                                                    int32_t* __restrict__ tile_md,
                                                                    int32_t* __restrict__ num_splits) {
+  griddep_launch_dependents();  // the decode kernel may start its set-up (it waits for this grid)
   __shared__ int s_payload;
   const int t = threadIdx.x;
   const int per = (U + kMetaThreads - 1) / kMetaThreads;
@@ -218,9 +220,84 @@ __global__ void __launch_bounds__(kMetaThreads) mla_metadata_kernel(const int32_
   }
 }
 
+// Up to kMetaSmemUnits units, the cost prefix C and the split prefix S live
+// in shared memory: the part boundaries are binary searches there, and every
+// output is written once. Larger problems use the same steps with C kept in
+// num_splits (global memory).
+constexpr int kMetaSmemUnits = 4096;
+
+__global__ void __launch_bounds__(kMetaThreads) mla_metadata_smem_kernel(const int32_t* __restrict__ seqlens,
+                                                                        int U, int upr, int topk, int parts,
+                                                                        int32_t* __restrict__ tile_md,
+                                                                        int32_t* __restrict__ num_splits) {
+  griddep_launch_dependents();  // the decode kernel may start its set-up (it waits for this grid)
+  __shared__ int32_t C[kMetaSmemUnits + 1];  // cost prefix
+  __shared__ int32_t S[kMetaSmemUnits + 1];  // split prefix
+  __shared__ int s_payload;
+  const int t = threadIdx.x;
+  const int per = (U + kMetaThreads - 1) / kMetaThreads;
+  const int u0 = min(U, t * per), u1 = min(U, u0 + per);
+  // 1. cost prefix C[0..U]
+  int my = 0, my_max = 0;
+  for (int u = u0; u < u1; ++u) {
+    const int n = unit_tiles(seqlens, u, upr, topk);
+    const int cost = n > 0 ? n + kSchedOverhead : 0;
+    C[u] = cost;
+    my += cost;
+    my_max = max(my_max, cost);
+  }
+  const int max_cost = block_max(my_max);
+  const int2 sc = block_exclusive_scan(my);
+  int c = sc.x;
+  for (int u = u0; u < u1; ++u) {
+    const int cost = C[u];
+    C[u] = c;
+    c += cost;
+  }
+  if (t == 0) {
+    C[U] = sc.y;
+    s_payload = choose_payload(sc.y, parts, max_cost);
+  }
+  __syncthreads();
+  const int total = sc.y, payload = s_payload;
+  // 2. split counts -> split prefix S[0..U] (also the num_splits output)
+  int mys = 0;
+  for (int u = u0; u < u1; ++u) {
+    const int n = C[u + 1] - C[u] - kSchedOverhead;  // tiles of unit u (cost 0: no tiles)
+    const int ns = n > 0 ? (int)((C[u] + kSchedOverhead + n - 1) / payload) - first_part_of(C[u], payload) + 1 : 0;
+    S[u] = ns;
+    mys += ns;
+  }
+  const int2 ss = block_exclusive_scan(mys);
+  int sp = ss.x;
+  for (int u = u0; u < u1; ++u) {
+    const int ns = S[u];
+    S[u] = sp;
+    num_splits[u] = sp;
+    sp += ns;
+  }
+  if (t == 0) {
+    S[U] = ss.y;
+    num_splits[U] = ss.y;
+  }
+  __syncthreads();
+  // 3. parts: boundaries by binary search on C, workspace index of the first piece
+  for (int p = t; p < parts; p += kMetaThreads) {
+    const int2 b = cost_to_tile(C, U, total, p * payload);
+    const int2 e = cost_to_tile(C, U, total, (p + 1) * payload);
+    const int ws = b.x < U ? p - first_part_of(C[b.x], payload) + S[b.x] : 0;
+    int32_t* md = tile_md + p * MLA_TILE_MD_INTS;
+    md[0] = b.x; md[1] = b.y; md[2] = e.x; md[3] = e.y;
+    md[4] = ws; md[5] = payload; md[6] = 0; md[7] = 0;
+  }
+}
+
 mla_status_t launch_metadata(const int32_t* seqlens, int U, int upr, int topk, int parts, int32_t* tile_md,
                              int32_t* num_splits, cudaStream_t stream) {
-  mla_metadata_kernel<<<1, kMetaThreads, 0, stream>>>(seqlens, U, upr, topk, parts, tile_md, num_splits);
+  if (U <= kMetaSmemUnits)
+    mla_metadata_smem_kernel<<<1, kMetaThreads, 0, stream>>>(seqlens, U, upr, topk, parts, tile_md, num_splits);
+  else
+    mla_metadata_kernel<<<1, kMetaThreads, 0, stream>>>(seqlens, U, upr, topk, parts, tile_md, num_splits);
   return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 

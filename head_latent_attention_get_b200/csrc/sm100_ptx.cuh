@@ -227,6 +227,13 @@ __device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster_addr) : "memory");
 }
+// Remote arrive without release semantics: it does not wait for this
+// thread's earlier memory operations (a release arrive after cp.async traffic
+// costs ~0.8K clk, this one ~0.1K). The caller orders the data it signals by
+// other means (an acquire of its completion, then a proxy fence).
+__device__ __forceinline__ void mbar_arrive_relaxed_cluster(uint32_t bar_cluster_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster_addr) : "memory");
+}
 // Counts `bytes` of transaction completion on a (possibly remote) mbarrier
 // without arriving. Relaxed: precede it with fence_acq_rel_cluster() when
 // data written by this thread must be visible to the waiter.
@@ -298,6 +305,18 @@ __device__ __forceinline__ void mma_commit_pair(uint64_t* bar) {
           smem_u32(bar)),
       "h"((uint16_t)3)
       : "memory");
+}
+
+// ---------------------------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialization may start while
+// the kernel before it in the stream is still running: it must wait here
+// before touching any global memory that kernel (or an earlier one) writes or
+// reads. Without that launch attribute the wait returns at once.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Lets the next kernel of the stream (if launched with the attribute) start
+// its blocks; its griddep_wait still waits for this whole grid to finish.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // ---------------------------------------------------------------- misc math

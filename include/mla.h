@@ -272,6 +272,45 @@ mla_status_t mla_decode_paged_noalloc(const mla_decode_args* args, mla_stream_t 
 mla_status_t mla_decode_sparse(const mla_decode_args* args, const int32_t* indices, int topk,
                                mla_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * The steps on either side of the attention ("deepseek-ai/FlashMLA"
+ * (agentlenshq), feature list: a fused kernel runs Q-norm, RoPE, the
+ * attention, the output-side conjugate RoPE and the final FP8 cast in one
+ * launch; the page names the steps, not their arithmetic). Query rows are
+ * [batch, s_q, h_q, d_qk] and output rows [batch, s_q, h_q, 512], row
+ * r = (b*s_q + i)*h_q + h; query token t = b*s_q + i. rope_cos/rope_sin:
+ * device fp32 [batch*s_q][32], cos/sin of the angle of RoPE pair p at query
+ * token t (the caller derives them from the token's position). Both calls
+ * are asynchronous on `stream`, allocate nothing and keep no state.
+ * ------------------------------------------------------------------------- */
+
+/* q_out = RMS-norm of each query row over its d_qk values times gamma,
+ * q / sqrt(mean(q^2) + eps) * gamma, then its last 64 dims (the RoPE part:
+ * 512..575 of a 576-dim row, 448..511 of a 512-dim row) rotated pair-wise,
+ * (x[2p], x[2p+1]) -> (x0 cos - x1 sin, x0 sin + x1 cos). Computed in fp32,
+ * rounded to bf16 (nearest even).
+ * q, q_out: device bf16 [rows][d_qk], 16-byte aligned; q_out may equal q.
+ * gamma: device fp32 [d_qk], 8-byte aligned. eps >= 0.
+ * Errors: INVALID_ARG for null or misaligned pointers, d_qk not 576 or 512,
+ * eps < 0, non-positive sizes; UNSUPPORTED above 2^31 rows; CUDA. */
+mla_status_t mla_q_norm_rope(const void* q, void* q_out, int batch, int s_q, int h_q, int d_qk,
+                             const float* gamma, float eps, const float* rope_cos, const float* rope_sin,
+                             mla_stream_t stream);
+
+/* Output epilogue: the output's RoPE part (the dims of V inside the last 64
+ * dims of d_qk: none when d_qk = 576, dims 448..511 when d_qk = 512) rotated
+ * back by the query token's angle, (x0 cos + x1 sin, x1 cos - x0 sin); then
+ * each 128-value tile cast to e4m3: scale = amax / 448 (1 when amax = 0),
+ * code = round-to-nearest-even(value / scale) saturated to +-448. Every
+ * product, sum and quotient is rounded once in fp32 (no contraction).
+ * out: device bf16 [rows][512], 16-byte aligned (the decode output).
+ * out_fp8: device uint8 [rows][512], 16-byte aligned; out_scale: device fp32
+ * [rows][4]. rope_cos/rope_sin may be NULL when d_qk = 576.
+ * Errors: INVALID_ARG for null or misaligned pointers, d_qk not 576 or 512,
+ * non-positive sizes; UNSUPPORTED above 2^31 rows; CUDA. */
+mla_status_t mla_out_rope_fp8(const void* out, int batch, int s_q, int h_q, int d_qk, const float* rope_cos,
+                              const float* rope_sin, void* out_fp8, float* out_scale, mla_stream_t stream);
+
 /* Split-KV combine alone (mla_decode_* call it already). For every unit u
  * with n = num_splits[u+1] - num_splits[u]:
  *   n >= 2: lse = ln sum_s exp(lse_s), out = sum_s exp(lse_s - lse) * o_s

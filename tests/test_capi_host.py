@@ -221,3 +221,22 @@ def test_host_scheduler_random_shapes_with_row_blocks():
         parts = int(rng.integers(1, 160))
         md, ns = host_schedule(lens, B, s_q, h_q, topk, parts)
         S.check_schedule(md, ns, lens, B, s_q, topk, parts, h_q=h_q)
+
+
+def test_pre_post_steps_validate_arguments_on_the_host():
+    """mla_q_norm_rope / mla_out_rope_fp8 reject bad arguments before any
+    launch (fake, aligned device pointers: nothing is dereferenced)."""
+    L = C.lib()
+    q, qo, g, cs, sn = 0x100000, 0x200000, 0x300000, 0x400000, 0x500000
+    assert L.mla_q_norm_rope(q, qo, 2, 1, 16, 600, g, 1e-6, cs, sn, None) == C.MLA_ERR_INVALID_ARG
+    assert L.mla_q_norm_rope(q + 8, qo, 2, 1, 16, 576, g, 1e-6, cs, sn, None) == C.MLA_ERR_INVALID_ARG
+    assert L.mla_q_norm_rope(q, qo, 2, 1, 16, 576, g + 4, 1e-6, cs, sn, None) == C.MLA_ERR_INVALID_ARG
+    assert L.mla_q_norm_rope(q, qo, 2, 1, 16, 576, None, 1e-6, cs, sn, None) == C.MLA_ERR_INVALID_ARG
+    assert L.mla_q_norm_rope(q, qo, 2, 1, 16, 576, g, -1.0, cs, sn, None) == C.MLA_ERR_INVALID_ARG
+    assert L.mla_q_norm_rope(q, qo, 0, 1, 16, 576, g, 1e-6, cs, sn, None) == C.MLA_ERR_INVALID_ARG
+    o, o8, sc = 0x100000, 0x200000, 0x300000
+    assert L.mla_out_rope_fp8(o, 2, 1, 16, 512, None, None, o8, sc, None) == C.MLA_ERR_INVALID_ARG
+    assert L.mla_out_rope_fp8(o, 2, 1, 16, 500, cs, sn, o8, sc, None) == C.MLA_ERR_INVALID_ARG
+    assert L.mla_out_rope_fp8(o, 2, 1, 16, 576, None, None, o8 + 4, sc, None) == C.MLA_ERR_INVALID_ARG
+    assert L.mla_out_rope_fp8(o, 2, 1, 16, 576, None, None, o8, sc + 2, None) == C.MLA_ERR_INVALID_ARG
+    assert L.mla_out_rope_fp8(None, 2, 1, 16, 576, None, None, o8, sc, None) == C.MLA_ERR_INVALID_ARG

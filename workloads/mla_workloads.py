@@ -351,3 +351,21 @@ def restrict(inp: DecodeInputs, requests) -> DecodeInputs:
         indices=None if inp.indices is None else inp.indices[requests].clone(),
         sink=inp.sink, q_scale=None if inp.q_scale is None else inp.q_scale[requests].clone(),
         kv_scale=None if inp.kv_scale is None else inp.kv_scale[pages].clone())
+
+
+def rope_tables(cache_seqlens, s_q: int, base: float = 10000.0):
+    """cos/sin [batch * s_q, 32] fp32 of the RoPE angles of every query token:
+    the s_q queries of request b sit at positions seqlen_b - s_q + i (the
+    request's last tokens), pair p turns by position * base^(-2p/64). Input
+    data for the query pre-step and the output epilogue (the caller supplies
+    the angles), not part of either computation."""
+    lens = np.asarray(cache_seqlens, dtype=np.float64).reshape(-1)
+    pos = lens[:, None] - s_q + np.arange(s_q)[None, :]
+    inv = base ** (-2.0 * np.arange(32) / 64.0)
+    ang = pos.reshape(-1, 1) * inv[None, :]
+    return (torch.from_numpy(np.cos(ang).astype(np.float32)), torch.from_numpy(np.sin(ang).astype(np.float32)))
+
+
+def norm_weight(d: int, seed: int) -> torch.Tensor:
+    """A seeded per-dimension RMS-norm weight, U(0.5, 1.5), fp32 [d]."""
+    return torch.from_numpy(_rng(seed).uniform(0.5, 1.5, size=d).astype(np.float32))
