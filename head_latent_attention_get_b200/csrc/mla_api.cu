@@ -45,6 +45,23 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The bf16 cache seen as [9 halves of 64 dims][rows][64 dims]: element
+// (e, t, h) at byte 1152 t + 128 h + 2 e (the row stride is larger than the
+// half stride; the driver accepts the order). A 64 x 64 x 2 box is the
+// 128-value-dim V slot of one page in a single copy, landing as two 8 KB
+// 128-B-swizzled halves, exactly the layout of two 64 x 64 boxes.
+bool make_map_v(CUtensorMap* m, const void* base, uint64_t rows) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {64, rows, (cuuint64_t)(kDqk / 64)};
+  cuuint64_t strides[2] = {(cuuint64_t)kDqk * 2, 128};
+  cuuint32_t box[3] = {64, 64, 2};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // {units per request, rows per unit}; rows 0 when the sizes are out of range.
@@ -96,16 +113,18 @@ mla_status_t run_decode(const mla_decode_args* a, const int32_t* indices, int to
   // and (bf16 paged cache only) the cache as [pages*64 tokens][576 dims];
   // boxes of 64 x 64 with 128-B swizzle. The FP8, NVFP4 and sparse modes read
   // the cache with cp.async and need no cache map.
-  CUtensorMap tq, tkv;
+  CUtensorMap tq, tkv, tv;
   std::memset(&tq, 0, sizeof(tq));
   std::memset(&tkv, 0, sizeof(tkv));
+  std::memset(&tv, 0, sizeof(tv));
   if (mode != kModeNvfp4 && !make_map(&tq, a->q, (uint64_t)U * rows, kDqk, kDqk * 2, 64, 64)) return MLA_ERR_CUDA;
   const int row_groups = (rows + kRowsPerCta - 1) / kRowsPerCta;
   // more than 64 rows on the BF16 cache (paged or sparse): one CTA pair per
   // part shares each cache tile between the two row halves
   const bool pair = row_groups == 2 && (mode == kModeBf16 || mode == kModeSparse);
   if (mode == kModeBf16 &&
-      !make_map(&tkv, a->kcache, (uint64_t)a->num_pages * kPage, kDqk, kDqk * 2, 64, 64))
+      (!make_map(&tkv, a->kcache, (uint64_t)a->num_pages * kPage, kDqk, kDqk * 2, 64, 64) ||
+       !make_map_v(&tv, a->kcache, (uint64_t)a->num_pages * kPage)))
     return MLA_ERR_CUDA;
   const WsLayout w = ws_layout(U, rows, a->num_sm_parts);
   char* ws = static_cast<char*>(a->workspace);
@@ -141,8 +160,8 @@ mla_status_t run_decode(const mla_decode_args* a, const int32_t* indices, int to
   p.q_scale = static_cast<const uint8_t*>(a->q_scale);
   p.kv_scale = static_cast<const uint8_t*>(a->kv_scale);
   const int rows_per_cta = rows < kRowsPerCta ? rows : kRowsPerCta;
-  const cudaError_t e = pair ? launch_decode_pair(tq, tkv, p, a->num_sm_parts, mode == kModeSparse, stream)
-                             : launch_decode(rows_per_cta, mode, tq, tkv, p, a->num_sm_parts, row_groups, stream);
+  const cudaError_t e = pair ? launch_decode_pair(tq, tkv, tv, p, a->num_sm_parts, mode == kModeSparse, stream)
+                             : launch_decode(rows_per_cta, mode, tq, tkv, tv, p, a->num_sm_parts, row_groups, stream);
   if (e != cudaSuccess) return MLA_ERR_CUDA;
   if (a->debug_flags & MLA_DEBUG_SKIP_COMBINE) return MLA_OK;
   return launch_combine(a->workspace, U, rows, a->num_sm_parts, a->num_splits, a->h_q, a->sink, a->out, a->lse,

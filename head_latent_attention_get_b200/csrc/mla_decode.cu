@@ -367,7 +367,7 @@ __device__ void gather_group(const DecodeParams& p, Ctrl* c, PieceIter& it, cons
 template <int NR, int MODE>
 __global__ void __launch_bounds__(MODE == kModeBf16 ? 256 : 256 + 2 * kGatherThreads, 1)
     mla_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
-                      const DecodeParams p) {
+                      const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
   using L = Smem<NR>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -402,7 +402,10 @@ __global__ void __launch_bounds__(MODE == kModeBf16 ? 256 : 256 + 2 * kGatherThr
   }
   if (warp == 0 && lane == 0 && MODE != kModeNvfp4) {
     tma_prefetch_desc(&tm_q);
-    if (MODE == kModeBf16) tma_prefetch_desc(&tm_kv);  // encoded only for the bf16 paged cache
+    if (MODE == kModeBf16) {  // encoded only for the bf16 paged cache
+      tma_prefetch_desc(&tm_kv);
+      tma_prefetch_desc(&tm_v);
+    }
   }
   if (warp == 1) {
     tmem_alloc(&c->tmem_base, kTmemCols);
@@ -511,8 +514,7 @@ __global__ void __launch_bounds__(MODE == kModeBf16 ? 256 : 256 + 2 * kGatherThr
             if (!timed_wait(c, &c->v_empty[slot], ((vc / kNV) & 1) ^ 1, p)) { stop = true; break; }
             mbar_arrive_expect_tx(&c->v_full[slot], kSlot);
             const int m = j >> 1, y = pg[j & 1] * kPage;
-            tma_load_2d(dst, &tm_kv, &c->v_full[slot], 128 * m, y);
-            tma_load_2d(dst + 8192, &tm_kv, &c->v_full[slot], 128 * m + 64, y);
+            tma_load_3d(dst, &tm_v, &c->v_full[slot], 0, y, 2 * m);  // value dims 128m.. in one copy
           }
         }
       }
@@ -814,25 +816,27 @@ __global__ void __launch_bounds__(MODE == kModeBf16 ? 256 : 256 + 2 * kGatherThr
 
 // ---------------------------------------------------------------- host side
 template <int NR, int MODE>
-static cudaError_t launch_one(const CUtensorMap& tq, const CUtensorMap& tkv, const DecodeParams& p, int parts,
+static cudaError_t launch_one(const CUtensorMap& tq, const CUtensorMap& tkv, const CUtensorMap& tv,
+                              const DecodeParams& p, int parts,
                               int row_groups, cudaStream_t stream) {
   constexpr int smem = Smem<NR>::total + 1024;
   auto kern = mla_decode_kernel<NR, MODE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   e = launch_pdl(kern, dim3(parts, row_groups), dim3(MODE == kModeBf16 ? 256 : 256 + 2 * kGatherThreads), smem,
-                 stream, tq, tkv, p);
+                 stream, tq, tkv, tv, p);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_decode(int rows_per_cta, int mode, const CUtensorMap& tq, const CUtensorMap& tkv,
-                          const DecodeParams& p, int parts, int row_groups, cudaStream_t stream) {
+                          const CUtensorMap& tv, const DecodeParams& p, int parts, int row_groups,
+                          cudaStream_t stream) {
 #define MLA_DISPATCH(NRV)                                                                         \
-  if (mode == kModeBf16) return launch_one<NRV, kModeBf16>(tq, tkv, p, parts, row_groups, stream); \
-  if (mode == kModeFp8) return launch_one<NRV, kModeFp8>(tq, tkv, p, parts, row_groups, stream);   \
-  if (mode == kModeSparse) return launch_one<NRV, kModeSparse>(tq, tkv, p, parts, row_groups, stream); \
-  if (mode == kModeNvfp4) return launch_one<NRV, kModeNvfp4>(tq, tkv, p, parts, row_groups, stream);   \
-  return launch_one<NRV, kModeFp8Sparse>(tq, tkv, p, parts, row_groups, stream);
+  if (mode == kModeBf16) return launch_one<NRV, kModeBf16>(tq, tkv, tv, p, parts, row_groups, stream); \
+  if (mode == kModeFp8) return launch_one<NRV, kModeFp8>(tq, tkv, tv, p, parts, row_groups, stream);   \
+  if (mode == kModeSparse) return launch_one<NRV, kModeSparse>(tq, tkv, tv, p, parts, row_groups, stream); \
+  if (mode == kModeNvfp4) return launch_one<NRV, kModeNvfp4>(tq, tkv, tv, p, parts, row_groups, stream);   \
+  return launch_one<NRV, kModeFp8Sparse>(tq, tkv, tv, p, parts, row_groups, stream);
   // <= 16 rows run in the 32-row kernel: the extra P^T rows are written as
   // zeros and their output rows are never stored
   if (rows_per_cta <= 32) { MLA_DISPATCH(32) }

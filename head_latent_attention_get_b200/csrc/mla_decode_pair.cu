@@ -174,7 +174,7 @@ __device__ __forceinline__ int sparse_slot_row(const DecodeParams& p, int unit, 
 template <bool SPARSE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SPARSE ? kThreadsSparse : kThreads, 1)
     mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
-                           const DecodeParams p) {
+                           const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + Smem::q;
@@ -212,7 +212,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SPARSE ? kThreadsSpa
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tm_q);
-    if (!SPARSE) tma_prefetch_desc(&tm_kv);  // the sparse path gathers rows with cp.async
+    if (!SPARSE) {  // the sparse path gathers rows with cp.async
+      tma_prefetch_desc(&tm_kv);
+      tma_prefetch_desc(&tm_v);
+    }
   }
   if (warp == 1) {
     tmem_alloc_pair(&c->tmem_base, kTmemCols);
@@ -299,8 +302,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SPARSE ? kThreadsSpa
               if (lane == 0 && pr.leader) mbar_arrive_expect_tx(&c->full[slot], 2 * kSlot);
               if (nv == kPage) {
                 if (lane == 0) {
-                  tma_load_2d_pair(dst, &tm_kv, bar, x0, pg * kPage);
-                  tma_load_2d_pair(dst + 8192, &tm_kv, bar, x0 + 64, pg * kPage);
+                  tma_load_3d_pair(dst, &tm_v, bar, 0, pg * kPage, x0 / 64);  // 128 value dims in one copy
                 }
               } else {
                 // keys past the request's end have zero probability, but their
@@ -309,8 +311,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SPARSE ? kThreadsSpa
                 if (nv > 0) {
                   if (lane == 0) {
                     mbar_arrive_expect_tx(&c->v_fix, kSlot);
-                    tma_load_2d(dst, &tm_kv, &c->v_fix, x0, pg * kPage);
-                    tma_load_2d(dst + 8192, &tm_kv, &c->v_fix, x0 + 64, pg * kPage);
+                    tma_load_3d(dst, &tm_v, &c->v_fix, 0, pg * kPage, x0 / 64);
                     ok = pwait(pr, &c->v_fix, fixc & 1, p);
                   }
                   ++fixc;
@@ -712,13 +713,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SPARSE ? kThreadsSpa
 
 }  // namespace pair
 
-cudaError_t launch_decode_pair(const CUtensorMap& tq, const CUtensorMap& tkv, const DecodeParams& p, int parts,
-                               bool sparse, cudaStream_t stream) {
+cudaError_t launch_decode_pair(const CUtensorMap& tq, const CUtensorMap& tkv, const CUtensorMap& tv,
+                               const DecodeParams& p, int parts, bool sparse, cudaStream_t stream) {
   constexpr int smem = pair::Smem::total + 1024;
   auto kern = sparse ? pair::mla_decode_pair_kernel<true> : pair::mla_decode_pair_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  e = launch_pdl(kern, dim3(2 * parts), dim3(sparse ? pair::kThreadsSparse : pair::kThreads), smem, stream, tq, tkv, p);
+  e = launch_pdl(kern, dim3(2 * parts), dim3(sparse ? pair::kThreadsSparse : pair::kThreads), smem, stream, tq, tkv, tv, p);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 

@@ -78,12 +78,16 @@ cudaError_t launch_pdl(void (*kern)(Params...), dim3 grid, dim3 block, size_t sm
   return cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...);
 }
 
+// tkv: the bf16 cache as [tokens][576] in 64 x 64 boxes; tv: the same bytes as
+// [64-dim halves of the row][tokens][64 dims] in 2 x 64 x 64 boxes (a V slot
+// of 128 value dims in one copy). Both unused by the FP8 / NVFP4 / sparse modes.
 cudaError_t launch_decode(int rows_per_cta, int mode, const CUtensorMap& tq, const CUtensorMap& tkv,
-                          const DecodeParams& p, int parts, int row_groups, cudaStream_t stream);
+                          const CUtensorMap& tv, const DecodeParams& p, int parts, int row_groups,
+                          cudaStream_t stream);
 // Units of more than 64 rows, BF16 cache (paged, or token-sparse when `sparse`):
 // CTA pairs (clusters of two), one per part.
-cudaError_t launch_decode_pair(const CUtensorMap& tq, const CUtensorMap& tkv, const DecodeParams& p, int parts,
-                               bool sparse, cudaStream_t stream);
+cudaError_t launch_decode_pair(const CUtensorMap& tq, const CUtensorMap& tkv, const CUtensorMap& tv,
+                               const DecodeParams& p, int parts, bool sparse, cudaStream_t stream);
 // How many CTA pairs of the pair kernel can be resident at once on the current device (0 if unknown).
 int max_pair_clusters();
 // Unit u reads seqlens[u / upr] (paged decoding; upr = units per request).
