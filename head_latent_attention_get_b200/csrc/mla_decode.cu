@@ -481,8 +481,8 @@ __global__ void __launch_bounds__(MODE == kModeBf16 ? 256 : 256 + 2 * kGatherThr
               uint8_t* dst = sK + slot * kSlot;
               if (!timed_wait(c, &c->k_empty[slot], ((kc / kNK) & 1) ^ 1, p)) { stop = true; break; }
               mbar_arrive_expect_tx(&c->k_full[slot], kSlot);
-              tma_load_2d(dst, &tm_kv, &c->k_full[slot], 64 * j, pa * kPage);
-              tma_load_2d(dst + 8192, &tm_kv, &c->k_full[slot], 64 * j, pb * kPage);
+              tma_load_2d_hint(dst, &tm_kv, &c->k_full[slot], 64 * j, pa * kPage, l2_policy_evict_last());
+              tma_load_2d_hint(dst + 8192, &tm_kv, &c->k_full[slot], 64 * j, pb * kPage, l2_policy_evict_last());
             }
           }
         }
@@ -514,7 +514,7 @@ __global__ void __launch_bounds__(MODE == kModeBf16 ? 256 : 256 + 2 * kGatherThr
             if (!timed_wait(c, &c->v_empty[slot], ((vc / kNV) & 1) ^ 1, p)) { stop = true; break; }
             mbar_arrive_expect_tx(&c->v_full[slot], kSlot);
             const int m = j >> 1, y = pg[j & 1] * kPage;
-            tma_load_3d(dst, &tm_v, &c->v_full[slot], 0, y, 2 * m);  // value dims 128m.. in one copy
+            tma_load_3d_hint(dst, &tm_v, &c->v_full[slot], 0, y, 2 * m, l2_policy_evict_first());
           }
         }
       }

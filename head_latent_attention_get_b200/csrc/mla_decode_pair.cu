@@ -275,8 +275,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SPARSE ? kThreadsSpa
               if (ok) {
                 const uint32_t bar = map_to_rank(smem_u32(&c->full[slot]), 0);
                 if (pr.leader) mbar_arrive_expect_tx(&c->full[slot], 2 * kSlot);
-                tma_load_2d_pair(dst, &tm_kv, bar, 64 * j, pa * kPage);
-                tma_load_2d_pair(dst + 8192, &tm_kv, bar, 64 * j, pb * kPage);
+                tma_load_2d_pair_hint(dst, &tm_kv, bar, 64 * j, pa * kPage, l2_policy_evict_last());
+                tma_load_2d_pair_hint(dst + 8192, &tm_kv, bar, 64 * j, pb * kPage, l2_policy_evict_last());
               }
             }
             ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -302,7 +302,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SPARSE ? kThreadsSpa
               if (lane == 0 && pr.leader) mbar_arrive_expect_tx(&c->full[slot], 2 * kSlot);
               if (nv == kPage) {
                 if (lane == 0) {
-                  tma_load_3d_pair(dst, &tm_v, bar, 0, pg * kPage, x0 / 64);  // 128 value dims in one copy
+                  tma_load_3d_pair_hint(dst, &tm_v, bar, 0, pg * kPage, x0 / 64, l2_policy_evict_first());
                 }
               } else {
                 // keys past the request's end have zero probability, but their

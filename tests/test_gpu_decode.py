@@ -173,3 +173,18 @@ def test_timeout_status_and_context_survives():
     ref_o, ref_l = G.oracle_for(inp)
     G.compare(out, lse, ref_o, ref_l, "after timeout")
     assert r2.status()[0] == C.MLA_OK
+
+
+def test_combine_strides_over_more_items_than_blocks():
+    """400 requests x 64 heads of mixed lengths: 400 units x 16 row chunks =
+    6400 combine items for a grid of at most 8 x 148 blocks, with many units
+    split across parts; every request against the oracle."""
+    rng = np.random.default_rng(404)
+    lens = [int(x) for x in rng.integers(1, 3000, size=400)]
+    w = _dense(batch=400, seqlens=lens, h_q=64, seed=404)
+    inp = W.make_inputs(w, poison_tail=True)
+    out, lse, r = G.run_gpu(inp)
+    ns = r.num_splits.cpu().numpy()
+    assert (np.diff(ns) > 1).sum() > 50            # many units are split
+    G.compare_full(inp, out, lse, "400 requests, 6400 combine items")
+    assert r.status()[0] == C.MLA_OK
