@@ -111,8 +111,9 @@ mla_status_t run_decode(const mla_decode_args* a, const int32_t* indices, int to
                                                : (fp8 ? kModeFp8 : kModeBf16);
   // Q rows of every unit (not NVFP4: its query is dequantised by the kernel),
   // and (bf16 paged cache only) the cache as [pages*64 tokens][576 dims];
-  // boxes of 64 x 64 with 128-B swizzle. The FP8, NVFP4 and sparse modes read
-  // the cache with cp.async and need no cache map.
+  // boxes of 64 x 64 with 128-B swizzle. The FP8 paged mode copies whole pages
+  // with cp.async.bulk, the NVFP4 and sparse modes gather rows with cp.async:
+  // none of them needs a cache map.
   CUtensorMap tq, tkv, tv;
   std::memset(&tq, 0, sizeof(tq));
   std::memset(&tkv, 0, sizeof(tkv));
@@ -160,8 +161,10 @@ mla_status_t run_decode(const mla_decode_args* a, const int32_t* indices, int to
   p.q_scale = static_cast<const uint8_t*>(a->q_scale);
   p.kv_scale = static_cast<const uint8_t*>(a->kv_scale);
   const int rows_per_cta = rows < kRowsPerCta ? rows : kRowsPerCta;
-  const cudaError_t e = pair ? launch_decode_pair(tq, tkv, tv, p, a->num_sm_parts, mode == kModeSparse, stream)
-                             : launch_decode(rows_per_cta, mode, tq, tkv, tv, p, a->num_sm_parts, row_groups, stream);
+  const cudaError_t e =
+      pair               ? launch_decode_pair(tq, tkv, tv, p, a->num_sm_parts, mode == kModeSparse, stream)
+      : mode == kModeFp8 ? launch_decode_fp8(rows_per_cta, tq, p, a->num_sm_parts, row_groups, stream)
+                         : launch_decode(rows_per_cta, mode, tq, tkv, tv, p, a->num_sm_parts, row_groups, stream);
   if (e != cudaSuccess) return MLA_ERR_CUDA;
   if (a->debug_flags & MLA_DEBUG_SKIP_COMBINE) return MLA_OK;
   return launch_combine(a->workspace, U, rows, a->num_sm_parts, a->num_splits, a->h_q, a->sink, a->out, a->lse,

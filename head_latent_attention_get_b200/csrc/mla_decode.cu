@@ -833,7 +833,6 @@ cudaError_t launch_decode(int rows_per_cta, int mode, const CUtensorMap& tq, con
                           cudaStream_t stream) {
 #define MLA_DISPATCH(NRV)                                                                         \
   if (mode == kModeBf16) return launch_one<NRV, kModeBf16>(tq, tkv, tv, p, parts, row_groups, stream); \
-  if (mode == kModeFp8) return launch_one<NRV, kModeFp8>(tq, tkv, tv, p, parts, row_groups, stream);   \
   if (mode == kModeSparse) return launch_one<NRV, kModeSparse>(tq, tkv, tv, p, parts, row_groups, stream); \
   if (mode == kModeNvfp4) return launch_one<NRV, kModeNvfp4>(tq, tkv, tv, p, parts, row_groups, stream);   \
   return launch_one<NRV, kModeFp8Sparse>(tq, tkv, tv, p, parts, row_groups, stream);

@@ -84,6 +84,10 @@ cudaError_t launch_pdl(void (*kern)(Params...), dim3 grid, dim3 block, size_t sm
 cudaError_t launch_decode(int rows_per_cta, int mode, const CUtensorMap& tq, const CUtensorMap& tkv,
                           const CUtensorMap& tv, const DecodeParams& p, int parts, int row_groups,
                           cudaStream_t stream);
+// FP8 paged cache: each page fetched by one bulk copy and converted once
+// (no cache tensor map).
+cudaError_t launch_decode_fp8(int rows_per_cta, const CUtensorMap& tq, const DecodeParams& p, int parts,
+                              int row_groups, cudaStream_t stream);
 // Units of more than 64 rows, BF16 cache (paged, or token-sparse when `sparse`):
 // CTA pairs (clusters of two), one per part.
 cudaError_t launch_decode_pair(const CUtensorMap& tq, const CUtensorMap& tkv, const CUtensorMap& tv,

@@ -104,9 +104,12 @@ def test_dense_shapes_vs_oracle(lens, s_q, h_q, causal):
     assert r.status()[0] == C.MLA_OK
 
 
-@pytest.mark.parametrize("parts", [1, 2, 7, 148])
-def test_split_counts_do_not_change_results(parts):
-    w = _dense(batch=3, seqlens=[900, 4000, 130], h_q=64, seed=77)
+@pytest.mark.parametrize("kv,parts", [("bf16", 1), ("bf16", 2), ("bf16", 7), ("bf16", 148),
+                                      ("fp8", 1), ("fp8", 3), ("fp8", 7), ("fp8", 148)])
+def test_split_counts_do_not_change_results(kv, parts):
+    """Pieces that start and end inside a request (odd page counts, a last
+    half tile, one-page requests) give the same results for any split count."""
+    w = _dense(batch=3, seqlens=[900, 4000, 130], h_q=64, seed=77, kv=kv)
     inp = W.make_inputs(w, poison_tail=True)
     out, lse, _ = G.run_gpu(inp, runner_kwargs={"num_sm_parts": parts})
     ref_o, ref_l = G.oracle_for(inp)
@@ -162,8 +165,12 @@ def test_bounds_status_without_fault():
     G.compare(out[1:], lse[1:], ref_o, ref_l, "unaffected request")
 
 
-def test_timeout_status_and_context_survives():
-    inp = W.make_inputs(W.get_workload("tiny"))
+@pytest.mark.parametrize("kv", ["bf16", "fp8"])
+def test_timeout_status_and_context_survives(kv):
+    """Scores withheld from the softmax: every bounded wait gives up, the
+    status word says so and the next call on the same context is exact (the
+    bf16 row-group kernel and the FP8 page kernel)."""
+    inp = W.make_inputs(_dense("tiny", kv=kv))
     _, _, r = G.run_gpu(inp, runner_kwargs={"timeout_ns": 20_000_000,
                                             "debug_flags": C.MLA_DEBUG_WITHHOLD_SCORES})
     code, bits = r.status()

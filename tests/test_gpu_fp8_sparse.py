@@ -75,7 +75,11 @@ def test_fp8_sparse_ignored_slots_are_bit_exact(h_q):
 
 
 @pytest.mark.parametrize("h_q", [64, 128])
-def test_fp8_all_positions_in_order_equal_fp8_dense(h_q):
+def test_fp8_all_positions_in_order_match_fp8_dense(h_q):
+    """Indices that list every position in order select the dense key set, so
+    the token-sparse path and the paged FP8 kernel must both reproduce the
+    oracle's dense result. The two kernels tile the keys differently (128-slot
+    tiles against 64-token pages), so they agree to rounding, not bitwise."""
     w = dataclasses.replace(W.get_workload("fp8"), batch=2, seqlens=[300, 190], h_q=h_q, seed=5)
     dense = W.make_inputs(w)
     idx = torch.full((2, 1, 320), -1, dtype=torch.int32)
@@ -84,8 +88,9 @@ def test_fp8_all_positions_in_order_equal_fp8_dense(h_q):
     sp = dataclasses.replace(dense, workload=dataclasses.replace(w, topk=320), indices=idx)
     do, dl, _ = _run(dense, num_sm_parts=1)
     so, sl, _ = _run(sp, num_sm_parts=1)
-    assert np.array_equal(so.view(np.uint32), do.view(np.uint32))
-    assert np.array_equal(sl.view(np.uint32), dl.view(np.uint32))
+    ref_o, ref_l = G.oracle_for(dense)
+    G.compare(do, dl, ref_o, ref_l, f"fp8 dense h_q={h_q}")
+    G.compare(so, sl, ref_o, ref_l, f"fp8 all positions h_q={h_q}")
 
 
 def test_fp8_sparse_full_size_every_request():
