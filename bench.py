@@ -59,11 +59,11 @@ def kernel_source_hash() -> str:
 def decode_kernel_name(w, rows: int) -> str:
     """The decode kernel the library launches for this workload: CTA pairs for
     units of 65-128 rows on the BF16 cache (paged or token-sparse), one CTA per
-    row group otherwise; the FP8 paged cache has a kernel of its own."""
+    row group otherwise; the FP8 and NVFP4 paged caches have a page kernel."""
     if w.kv == "bf16" and rows > 64:
         return "mla_decode_pair_kernel"
-    if w.kv == "fp8" and w.topk == 0:
-        return "mla_decode_fp8_kernel"
+    if w.kv in ("fp8", "nvfp4") and w.topk == 0:
+        return "mla_decode_page_kernel"
     return "mla_decode_kernel"
 
 

@@ -111,9 +111,9 @@ mla_status_t run_decode(const mla_decode_args* a, const int32_t* indices, int to
                                                : (fp8 ? kModeFp8 : kModeBf16);
   // Q rows of every unit (not NVFP4: its query is dequantised by the kernel),
   // and (bf16 paged cache only) the cache as [pages*64 tokens][576 dims];
-  // boxes of 64 x 64 with 128-B swizzle. The FP8 paged mode copies whole pages
-  // with cp.async.bulk, the NVFP4 and sparse modes gather rows with cp.async:
-  // none of them needs a cache map.
+  // boxes of 64 x 64 with 128-B swizzle. The FP8 and NVFP4 paged modes copy
+  // whole pages with cp.async.bulk, the sparse modes gather rows with
+  // cp.async: none of them needs a cache map.
   CUtensorMap tq, tkv, tv;
   std::memset(&tq, 0, sizeof(tq));
   std::memset(&tkv, 0, sizeof(tkv));
@@ -163,7 +163,8 @@ mla_status_t run_decode(const mla_decode_args* a, const int32_t* indices, int to
   const int rows_per_cta = rows < kRowsPerCta ? rows : kRowsPerCta;
   const cudaError_t e =
       pair               ? launch_decode_pair(tq, tkv, tv, p, a->num_sm_parts, mode == kModeSparse, stream)
-      : mode == kModeFp8 ? launch_decode_fp8(rows_per_cta, tq, p, a->num_sm_parts, row_groups, stream)
+      : (mode == kModeFp8 || mode == kModeNvfp4)
+          ? launch_decode_page(mode, rows_per_cta, tq, p, a->num_sm_parts, row_groups, stream)
                          : launch_decode(rows_per_cta, mode, tq, tkv, tv, p, a->num_sm_parts, row_groups, stream);
   if (e != cudaSuccess) return MLA_ERR_CUDA;
   if (a->debug_flags & MLA_DEBUG_SKIP_COMBINE) return MLA_OK;
@@ -219,7 +220,7 @@ mla_status_t mla_get_metadata(const int32_t* cache_seqlens, int batch, int s_q, 
   if (h_kv != 1) return MLA_ERR_UNSUPPORTED;
   const Geometry g = geometry_of(s_q, h_q, h_kv, topk);
   if (g.rows <= 0 || (long long)batch * g.units_per_req > 0x7fffffff) return MLA_ERR_UNSUPPORTED;
-  return launch_metadata(cache_seqlens, batch * g.units_per_req, g.units_per_req, topk, num_sm_parts, tile_md,
+  return launch_metadata(cache_seqlens, batch * g.units_per_req, g.units_per_req, topk, num_sm_parts, g.rows, tile_md,
                          num_splits, reinterpret_cast<cudaStream_t>(stream));
 }
 

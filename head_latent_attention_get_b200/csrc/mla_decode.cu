@@ -3,8 +3,8 @@
 // Computes, per work unit (a block of <= 128 query rows of a request, or
 // (request, query token) when sparse), softmax(scale * Q K^T) V over the
 // unit's keys, with K = whole 576-dim latent row and V = its first 512 dims
-// (NVFP4: a 512-value row that is both) ("[flashinfer] ... NVFP4 DeepSeek-V4
-// decoding", README section: one latent row per token is both K and V;
+// ("[flashinfer] ... NVFP4 DeepSeek-V4 decoding", README section: one latent
+// row per token is both K and V;
 // FlashMLA-ETAP summary, core mechanism: S = QK^T, P = softmax(S), O = PV).
 //
 // One CTA = one scheduler part x one group of <= 64 query rows. Per tile of
@@ -24,14 +24,16 @@
 // the PV product rather than held across the softmax, which keeps the rings
 // deep enough to cover the load latency.
 //
-// Warp roles (256 threads for the bf16 paged cache; 512 with the FP8 or NVFP4
-// cache or sparse indices):
+// Serves the BF16 paged cache and token-sparse indices over the BF16 or FP8
+// cache (the FP8 and NVFP4 paged caches have the page kernel).
+//
+// Warp roles (256 threads for the bf16 paged cache; 512 with sparse indices):
 //   0 Q (and, bf16 paged, K slices) via TMA   1 S issuer (+ TMEM alloc)
 //   2 O issuer                                 3 V slots via TMA (bf16 paged)
 //   4-7 softmax + epilogue (row r = 16*(warp-4) + lane, lanes 0-15)
-//   8-11 K gather warps, 12-15 V gather warps (FP8 / NVFP4 / sparse): cp.async
-//       copies software-pipelined two slots deep; FP8 and NVFP4 codes are
-//       converted to bf16 in place.
+//   8-11 K gather warps, 12-15 V gather warps (sparse): cp.async copies
+//       software-pipelined two slots deep; FP8 codes are converted to bf16 in
+//       place.
 // Every mbarrier wait is bounded; on timeout the CTA records
 // MLA_DEVICE_STATUS_TIMEOUT, stops issuing work, waits (bounded) for its own
 // copies in flight and exits normally. Every ring has exactly one producer
@@ -54,9 +56,6 @@ constexpr int kTmemS = 256;            // S buffers at columns 256 and 384
 constexpr float kRescaleLog2 = 8.0f;   // rescale O only when the max grows by > 2^8
 static_assert(kLag < kNK && kLag < kNV, "a gather group must retire a slot before reusing it");
 
-// K slices of 64 dims per tile: 576-dim rows (512 latent + 64 RoPE) or the
-// 512-value NVFP4 rows.
-__host__ __device__ constexpr int k_slices(int mode) { return mode == kModeNvfp4 ? 8 : 9; }
 
 template <int NR>
 struct Smem {
@@ -102,14 +101,14 @@ __device__ __forceinline__ bool group_sync(Ctrl* c, uint64_t* bar, uint32_t& pha
 }
 
 // ============================================================================ gather groups
-// FP8, NVFP4 and sparse modes: four warps fill the K ring and four the V ring with
+// Sparse modes: four warps fill the K ring and four the V ring with
 // 16-byte cp.async copies. Warp lw of a group owns a quarter of every slot's
 // rows (K: tile rows 32lw..32lw+31; V: page rows 16lw..16lw+15), lane t the
 // source row of one of them; the copies put 4-16 lanes on each row (row
 // pointers by shuffle), FP8 codes are converted in place with four lanes per
 // row. Each warp issues a slot's copies, commits them as one group and retires
 // the slot it issued kLag slots earlier: wait for that group, convert it
-// (FP8, NVFP4), fence the generic-proxy writes for the tensor core, and one
+// (FP8), fence the generic-proxy writes for the tensor core, and one
 // lane arrives on the slot's full barrier (count: 4 warps).
 constexpr int kGatherWarps = 4;
 constexpr int kGatherThreads = 32 * kGatherWarps;
@@ -133,54 +132,7 @@ template <int MODE, bool KGROUP>
 __device__ __forceinline__ void retire_slot(const GatherRing& g, int seq, int lw, int t) {
   const int slot = seq % g.nslots;
   uint8_t* s = g.base + slot * kSlot;
-  if (MODE == kModeNvfp4) {
-    __syncwarp();  // every lane's copies of this slot are complete and visible
-    if (KGROUP) {  // slice j: codes in bytes [0,32), the 16-byte scale chunk 16*(j/4).. in [32,48) of each row
-      const int j = seq % 8;
-      uint2 cw[4];
-      uint32_t sb[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int r = 32 * lw + 8 * i + (t >> 2), cc = t & 3;  // values 16cc..16cc+15 of the slice
-        cw[i] = *reinterpret_cast<const uint2*>(s + r * 128 + 8 * cc);
-        sb[i] = s[r * 128 + 32 + 4 * (j & 3) + cc];
-      }
-      __syncwarp();
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int r = 32 * lw + 8 * i + (t >> 2), cc = t & 3;
-        uint4 lo, hi;
-        dequant_nvfp4_16(cw[i], sb[i], lo, hi);
-        *reinterpret_cast<uint4*>(sw128(s, r, 2 * cc)) = lo;
-        *reinterpret_cast<uint4*>(sw128(s, r, 2 * cc + 1)) = hi;
-      }
-    } else {  // V slot: codes (64 B) and the scale chunk 16*(m/2).. in the half-0 row
-      const int m = (seq >> 1) & 3;
-      uint4 cw[2];
-      uint32_t sb[2][2];
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const int r = 16 * lw + 8 * i + (t >> 2), c4 = t & 3;  // values 32c4..32c4+31 of the 128
-        cw[i] = *reinterpret_cast<const uint4*>(s + r * 128 + 16 * c4);
-        sb[i][0] = s[r * 128 + 64 + 8 * (m & 1) + 2 * c4];
-        sb[i][1] = s[r * 128 + 64 + 8 * (m & 1) + 2 * c4 + 1];
-      }
-      __syncwarp();
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const int r = 16 * lw + 8 * i + (t >> 2), c4 = t & 3;
-        uint8_t* half = s + (c4 >> 1) * 8192;
-        const int c0 = 4 * (c4 & 1);
-        uint4 lo, hi;
-        dequant_nvfp4_16(make_uint2(cw[i].x, cw[i].y), sb[i][0], lo, hi);
-        *reinterpret_cast<uint4*>(sw128(half, r, c0)) = lo;
-        *reinterpret_cast<uint4*>(sw128(half, r, c0 + 1)) = hi;
-        dequant_nvfp4_16(make_uint2(cw[i].z, cw[i].w), sb[i][1], lo, hi);
-        *reinterpret_cast<uint4*>(sw128(half, r, c0 + 2)) = lo;
-        *reinterpret_cast<uint4*>(sw128(half, r, c0 + 3)) = hi;
-      }
-    }
-  } else if (mode_fp8(MODE)) {
+  if (mode_fp8(MODE)) {
     __syncwarp();  // every lane's copies of this slot are complete and visible
     if (KGROUP) {
       const int j = seq % 9;
@@ -237,23 +189,16 @@ __device__ __forceinline__ void retire_slot(const GatherRing& g, int seq, int lw
   if (t == 0) mbar_arrive(&g.full[slot]);  // one arrival per warp (a per-thread one costs more)
 }
 
-// Source row of tile-relative token tt of tile k (FP8 record, or bf16 cache
-// row; ok = 0 for an ignored sparse slot, whose copies zero-fill: codes and
-// scales 0 dequantise to 0 as well).
+// Source row of tile-relative slot tt of index tile k (bf16 cache row or FP8
+// record; the gather warps run only with token-sparse indices; ok = 0 for an
+// ignored slot, whose copies zero-fill: codes and scales
+// 0 dequantise to 0 as well).
 template <int MODE, bool KGROUP>
-__device__ __forceinline__ const uint8_t* gather_src(const DecodeParams& p, int unit, int req, int npg, int k, int tt,
-                                                     uint32_t& ok) {
-  if (mode_sparse(MODE)) {
-    const int row = sparse_row(p, unit, k * kTile + tt, KGROUP);
-    ok = row >= 0 ? 16u : 0u;
-    const size_t rb = MODE == kModeSparse ? (size_t)kDqk * 2 : (size_t)kFp8RecordBytes;
-    return static_cast<const uint8_t*>(p.kcache) + (size_t)(row >= 0 ? row : 0) * rb;
-  }
-  int pg = page_of(p, req, 2 * k + (tt >> 6), npg);
-  if (pg < 0) pg = page_of(p, req, 2 * k, npg);  // half tile: page A again (keys masked, values zero-filled later)
-  ok = 16u;
-  const size_t rb = MODE == kModeNvfp4 ? (size_t)kNvfp4RowBytes : (size_t)kFp8RecordBytes;
-  return p.kcache_fp8 + ((size_t)pg * kPage + (tt & 63)) * rb;
+__device__ __forceinline__ const uint8_t* gather_src(const DecodeParams& p, int unit, int k, int tt, uint32_t& ok) {
+  const int row = sparse_row(p, unit, k * kTile + tt, KGROUP);
+  ok = row >= 0 ? 16u : 0u;
+  const size_t rb = MODE == kModeSparse ? (size_t)kDqk * 2 : (size_t)kFp8RecordBytes;
+  return static_cast<const uint8_t*>(p.kcache) + (size_t)(row >= 0 ? row : 0) * rb;
 }
 
 template <int MODE, bool KGROUP>
@@ -264,8 +209,6 @@ __device__ void gather_group(const DecodeParams& p, Ctrl* c, PieceIter& it, cons
   Piece pc;
   while (!stop && it.next(pc)) {
     const int unit = pc.unit;
-    const int req = unit_req(p, unit);
-    const int npg = mode_sparse(MODE) ? 0 : (p.seqlens[req] + kPage - 1) / kPage;
     for (int k = pc.t0; k < pc.t1 && !stop; ++k) {
       // K: lane t owns tile row 32lw + t; V: lane t (< 16) owns row 16lw + t
       // of page h, i.e. tile row 64h + 16lw + t
@@ -274,52 +217,30 @@ __device__ void gather_group(const DecodeParams& p, Ctrl* c, PieceIter& it, cons
       const uint8_t* srcV0 = nullptr;
       const uint8_t* srcV1 = nullptr;
       if (KGROUP) {
-        srcK = gather_src<MODE, KGROUP>(p, unit, req, npg, k, 32 * lw + t, ok);
+        srcK = gather_src<MODE, KGROUP>(p, unit, k, 32 * lw + t, ok);
       } else {
-        srcV0 = gather_src<MODE, KGROUP>(p, unit, req, npg, k, 16 * lw + (t & 15), ok0);
-        srcV1 = gather_src<MODE, KGROUP>(p, unit, req, npg, k, 64 + 16 * lw + (t & 15), ok1);
+        srcV0 = gather_src<MODE, KGROUP>(p, unit, k, 16 * lw + (t & 15), ok0);
+        srcV1 = gather_src<MODE, KGROUP>(p, unit, k, 64 + 16 * lw + (t & 15), ok1);
       }
-      const int slots_per_tile = KGROUP ? k_slices(MODE) : 8;
+      const int slots_per_tile = KGROUP ? 9 : 8;
       for (int j = 0; j < slots_per_tile; ++j, ++seq) {
         const int slot = seq % g.nslots;
         uint8_t* s = g.base + slot * kSlot;
         if (!timed_wait(c, &g.empty[slot], ((seq / g.nslots) & 1) ^ 1, p)) { stop = true; break; }
-        if (MODE == kModeNvfp4) {
-          // row pointers: codes (256 B per row) and scales (32 B per row, the
-          // row's byte offset / 8 into the scale array)
-          if (KGROUP) {  // slice j: 32 code bytes (2 lanes per row) + a 16-byte scale chunk
-            const uint8_t* srcS = p.kv_scale + ((srcK - p.kcache_fp8) >> 3);
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-              const int r = 16 * i + (t >> 1), ch = t & 1;
-              cp_async16(s + (32 * lw + r) * 128 + 16 * ch, shfl_ptr(srcK, r) + 32 * j + 16 * ch, 16u);
-            }
-            cp_async16(s + (32 * lw + t) * 128 + 32, srcS + 16 * (j >> 2), 16u);
-          } else {  // V slot j: 64 code bytes of value group m (4 lanes per row) + a scale chunk
-            const int m = j >> 1;
-            const uint8_t* sv = (j & 1) ? srcV1 : srcV0;
-            const uint8_t* srcS = p.kv_scale + ((sv - p.kcache_fp8) >> 3);
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-              const int r = 8 * i + (t >> 2), ch = t & 3;
-              cp_async16(s + (16 * lw + r) * 128 + 16 * ch, shfl_ptr(sv, r) + 64 * m + 16 * ch, 16u);
-            }
-            if (t < 16) cp_async16(s + (16 * lw + t) * 128 + 64, srcS + 16 * (m >> 1), 16u);
-          }
-        } else if (KGROUP) {
+        if (KGROUP) {
           if (MODE == kModeSparse || j == 8) {  // bf16 128-B row slice: 8 lanes per row
             const int off = MODE == kModeSparse ? 128 * j : 528;
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
               const int r = 4 * i + (t >> 3), ch = t & 7;
-              const uint32_t nb = mode_sparse(MODE) ? __shfl_sync(0xffffffffu, ok, r) : 16u;
+              const uint32_t nb = __shfl_sync(0xffffffffu, ok, r);
               cp_async16(sw128(s, 32 * lw + r, ch), shfl_ptr(srcK, r) + off + 16 * ch, nb);
             }
           } else {  // FP8 latent slice j: codes (64 B, 4 lanes per row) and scales, converted at retire
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const int r = 8 * i + (t >> 2), cc = t & 3;
-              const uint32_t nb = mode_sparse(MODE) ? __shfl_sync(0xffffffffu, ok, r) : 16u;
+              const uint32_t nb = __shfl_sync(0xffffffffu, ok, r);
               cp_async16(s + (32 * lw + r) * 128 + 16 * cc, shfl_ptr(srcK, r) + 64 * j + 16 * cc, nb);
             }
             cp_async16(s + (32 * lw + t) * 128 + 64, srcK + 512, ok);
@@ -339,7 +260,7 @@ __device__ void gather_group(const DecodeParams& p, Ctrl* c, PieceIter& it, cons
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const int r = 4 * i + (t >> 3), ch = t & 7;
-              const uint32_t nb = mode_sparse(MODE) ? __shfl_sync(0xffffffffu, okv, r) : 16u;
+              const uint32_t nb = __shfl_sync(0xffffffffu, okv, r);
               cp_async16(s + (16 * lw + r) * 128 + 16 * ch, shfl_ptr(sv, r) + 128 * m + 16 * ch, nb);
             }
             if (t < 16) cp_async16(s + 8192 + (16 * lw + t) * 128, sv + 512, okv);
@@ -400,7 +321,7 @@ __global__ void __launch_bounds__(MODE == kModeBf16 ? 256 : 256 + 2 * kGatherThr
     c->rescale_flag[1] = 0;
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0 && MODE != kModeNvfp4) {
+  if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tm_q);
     if (MODE == kModeBf16) {  // encoded only for the bf16 paged cache
       tma_prefetch_desc(&tm_kv);
@@ -426,40 +347,6 @@ __global__ void __launch_bounds__(MODE == kModeBf16 ? 256 : 256 + 2 * kGatherThr
     int kc = 0, pi = 0, q_issued = 0;
     bool stop = false;
     while (!stop && it.next(pc)) {
-      if (MODE == kModeNvfp4) {
-        // Q rows dequantised by this warp: lane l converts value block l
-        // (dims 16l..16l+15) of each row into box l/4, chunks 2(l%4), 2(l%4)+1;
-        // rows past this CTA's rows are zero
-        if (lane == 0 && !timed_wait(c, &c->q_empty, (pi & 1) ^ 1, p)) stop = true;
-        stop = __shfl_sync(0xffffffffu, stop ? 1 : 0, 0) != 0;
-        if (stop) break;
-        const size_t qrow0 = (size_t)pc.unit * p.rows + row0;
-        uint8_t* box = sQ + (lane >> 2) * 8192;
-#pragma unroll 1
-        for (int r0 = 0; r0 < kRowsPerCta; r0 += 8) {
-          uint2 cw[8];
-          uint32_t sb[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const bool live = r0 + i < rows_here;
-            const size_t qr = qrow0 + (live ? r0 + i : 0);
-            cw[i] = live ? *reinterpret_cast<const uint2*>(p.q_nvfp4 + qr * kNvfp4RowBytes + 8 * lane) : make_uint2(0, 0);
-            sb[i] = live ? p.q_scale[qr * kNvfp4ScaleBytes + lane] : 0u;
-          }
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            uint4 lo, hi;
-            dequant_nvfp4_16(cw[i], sb[i], lo, hi);
-            *reinterpret_cast<uint4*>(sw128(box, r0 + i, 2 * (lane & 3))) = lo;
-            *reinterpret_cast<uint4*>(sw128(box, r0 + i, 2 * (lane & 3) + 1)) = hi;
-          }
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&c->q_full);
-        ++pi;
-        continue;
-      }
       if (lane == 0) {
         if (!timed_wait(c, &c->q_empty, (pi & 1) ^ 1, p)) {
           stop = true;
@@ -490,7 +377,7 @@ __global__ void __launch_bounds__(MODE == kModeBf16 ? 256 : 256 + 2 * kGatherThr
       stop = __shfl_sync(0xffffffffu, stop ? 1 : 0, 0) != 0;
       ++pi;
     }
-    if (lane == 0 && MODE != kModeNvfp4) {
+    if (lane == 0) {
       if (q_issued > 0) mbar_wait(&c->q_full, (uint32_t)((q_issued - 1) & 1), p.timeout_ns);
       if (MODE == kModeBf16) drain_issued(c->k_full, kNK, kc, p.timeout_ns);
     }
@@ -543,7 +430,7 @@ __global__ void __launch_bounds__(MODE == kModeBf16 ? 256 : 256 + 2 * kGatherThr
           if (!timed_wait(c, &c->s_empty[b], ((gt >> 1) & 1) ^ 1, p)) { stop = true; }
           tc_fence_after();
           const uint32_t d = tmem + kTmemS + 128 * b;
-          for (int j = 0; j < k_slices(MODE) && !stop; ++j, ++kc) {
+          for (int j = 0; j < 9 && !stop; ++j, ++kc) {
             const int slot = kc % kNK;
             if (!timed_wait(c, &c->k_full[slot], (kc / kNK) & 1, p)) { stop = true; break; }
             tc_fence_after();
@@ -834,7 +721,6 @@ cudaError_t launch_decode(int rows_per_cta, int mode, const CUtensorMap& tq, con
 #define MLA_DISPATCH(NRV)                                                                         \
   if (mode == kModeBf16) return launch_one<NRV, kModeBf16>(tq, tkv, tv, p, parts, row_groups, stream); \
   if (mode == kModeSparse) return launch_one<NRV, kModeSparse>(tq, tkv, tv, p, parts, row_groups, stream); \
-  if (mode == kModeNvfp4) return launch_one<NRV, kModeNvfp4>(tq, tkv, tv, p, parts, row_groups, stream);   \
   return launch_one<NRV, kModeFp8Sparse>(tq, tkv, tv, p, parts, row_groups, stream);
   // <= 16 rows run in the 32-row kernel: the extra P^T rows are written as
   // zeros and their output rows are never stored

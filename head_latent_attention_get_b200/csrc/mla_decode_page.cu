@@ -1,28 +1,33 @@
-// MLA decode over the FP8 paged cache for sm_100a: every page is fetched once
-// by one bulk copy and converted once.
+// MLA decode over a quantised paged cache (FP8 records or NVFP4 rows) for
+// sm_100a: every page is fetched once by bulk copies and converted once.
 //
-// Each cached token is one 656-byte record: 512 e4m3 latent codes, four fp32
-// scales (one per 128 codes) and the 64 RoPE dims in bf16 ("deepseek-ai/
-// FlashMLA", technical details: an FP8 KV cache dequantised on the fly). The
-// 64 records of a page are one contiguous 41,984-byte run. One
-// cp.async.bulk puts that run at the tail of a 72 KB page slot, and eight
-// converter warps expand it in place into nine 64-token x 64-dim bf16 slices
-// (128-B swizzled), x = bf16(f32(e4m3) * scale). The same slices feed both
-// products of the page:
-//   S    = Q K^T     tcgen05 M=64 rows x N=64 tokens x K=576 (slices 0-8 as
-//                    the K-major B operand)
+// FP8: each cached token is one 656-byte record of 512 e4m3 latent codes,
+// four fp32 scales (one per 128 codes) and the 64 RoPE dims in bf16
+// ("deepseek-ai/FlashMLA", technical details: an FP8 KV cache dequantised on
+// the fly); x = bf16(f32(e4m3) * scale). The 64 records of a page are one
+// contiguous 41,984-byte run.
+// NVFP4 ("[flashinfer] ... NVFP4 DeepSeek-V4 decoding", README: one 512-value
+// row per token is both K and V, E2M1 codes two per byte with a UE4M3 scale
+// per 16 values, and an NVFP4 query): a page is 16 KB of codes and 2 KB of
+// scales, each contiguous; x = e2m1 * ue4m3, exact in bf16.
+// Bulk copies put a page's bytes at the tail of a 72 KB page slot, and eight
+// converter warps expand them in place into 64-token x 64-dim bf16 slices
+// (128-B swizzled): nine for FP8 (576 dims), eight for NVFP4 (512). The same
+// slices feed both products of the page:
+//   S    = Q K^T     tcgen05 M=64 rows x N=64 tokens x K=576 or 512 (the
+//                    slices as the K-major B operand)
 //   O^T += V^T P^T   M=128 value dims (slices 2m and 2m+1, read MN-major) x
 //                    N=rows x K=64 tokens
-// so no record crosses from L2 twice and none is converted twice. Q takes
-// 72 KB, which leaves room for two page slots: one page is fetched and
-// converted while the other is multiplied.
+// so no cache byte crosses from L2 twice and none is converted twice. Q takes
+// 72 KB (64 KB for NVFP4), which leaves room for two page slots: one page is
+// fetched and converted while the other is multiplied.
 //
 // Warp roles (512 threads):
-//   0 Q (TMA) and the page copies     1 S issuer (+ TMEM alloc)
-//   2 O issuer                        3 idle
+//   0 Q (TMA, or dequantised from NVFP4 by the warp) and the page copies
+//   1 S issuer (+ TMEM alloc)          2 O issuer          3 idle
 //   4-7 softmax + epilogue (row r = 16*(warp-4) + lane, lanes 0-15)
 //   8-15 converters: thread (token 8*(warp-8) + lane%8, quarter lane/8 of the
-//        record's codes)
+//        token's latent values)
 // The softmax, the lazily rescaled O^T accumulator and the split epilogue are
 // those of the bf16 row-group kernel, on 64-token pages. Every wait is
 // bounded; on a timeout the CTA records MLA_DEVICE_STATUS_TIMEOUT, stops
@@ -36,21 +41,26 @@
 namespace mla {
 namespace {
 
-constexpr int kQB = 9 * 8192;                            // 64 rows x 576 dims
-constexpr int kSlotB = 9 * 8192;                         // one page: nine 64 x 64 bf16 slices
-constexpr int kRawB = kPage * kFp8RecordBytes;           // 41,984 bytes of records
-constexpr int kRawOff = kSlotB - kRawB;                  // records land at the slot's tail
+constexpr int kSlotB = 9 * 8192;                         // one page: up to nine 64 x 64 bf16 slices
+constexpr int kQMax = 9 * 8192;                          // 64 rows x 576 dims
+// 64-dim slices per row, raw page bytes, where they land in the slot
+__host__ __device__ constexpr int slices_of(int mode) { return mode == kModeNvfp4 ? 8 : 9; }
+__host__ __device__ constexpr int raw_bytes(int mode) {
+  return mode == kModeNvfp4 ? kPage * (kNvfp4RowBytes + kNvfp4ScaleBytes) : kPage * kFp8RecordBytes;
+}
+__host__ __device__ constexpr int raw_off(int mode) { return kSlotB - raw_bytes(mode); }
 constexpr int kCvWarps = 8;
 constexpr int kThreads = 256 + 32 * kCvWarps;
 constexpr int kTmemCols = 512;
 constexpr int kTmemS = 256;                              // S buffers at columns 256 and 320
 constexpr float kRescaleLog2 = 8.0f;                     // rescale O only when the max grows by > 2^8
-static_assert(kRawOff % 16 == 0 && kRawB % 16 == 0, "bulk copy alignment");
+static_assert(raw_off(kModeFp8) % 16 == 0 && raw_bytes(kModeFp8) % 16 == 0, "bulk copy alignment");
+static_assert(raw_off(kModeNvfp4) % 16 == 0 && (kPage * kNvfp4RowBytes) % 16 == 0, "bulk copy alignment");
 
 template <int NR>
 struct Smem {
   static constexpr int q = 0;
-  static constexpr int slot = q + kQB;
+  static constexpr int slot = q + kQMax;
   static constexpr int pt = slot + 2 * kSlotB;
   static constexpr int pt_bytes = NR * 128;              // P^T: [NR rows][64 tokens] bf16
   static constexpr int ctrl = pt + pt_bytes;
@@ -91,9 +101,12 @@ __device__ __forceinline__ bool group_sync(Ctrl* c, uint64_t* bar, uint32_t& pha
 // Logical pages [2*t0, end) of a piece: its 128-token tiles, cut at the request's last page.
 __device__ __forceinline__ int piece_page_end(const Piece& pc, int npg) { return min(2 * pc.t1, npg); }
 
-template <int NR>
+template <int NR, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
-    mla_decode_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const DecodeParams p) {
+    mla_decode_page_kernel(const __grid_constant__ CUtensorMap tm_q, const DecodeParams p) {
+  constexpr int kSl = slices_of(MODE);
+  constexpr int kRawB = raw_bytes(MODE);
+  constexpr int kRawOff = raw_off(MODE);
   using L = Smem<NR>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -129,7 +142,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     c->rescale_flag[1] = 0;
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) tma_prefetch_desc(&tm_q);
+  if (warp == 0 && lane == 0 && MODE != kModeNvfp4) tma_prefetch_desc(&tm_q);
   if (warp == 1) {
     tmem_alloc(&c->tmem_base, kTmemCols);
     tmem_relinquish();
@@ -149,25 +162,61 @@ __global__ void __launch_bounds__(kThreads, 1)
     int gp = 0, pi = 0, q_issued = 0;
     bool stop = false;
     while (!stop && it.next(pc)) {
-      if (lane == 0) {
-        if (!timed_wait(c, &c->q_empty, (pi & 1) ^ 1, p)) {
-          stop = true;
-        } else {
-          mbar_arrive_expect_tx(&c->q_full, kQB);
-          const int qy = pc.unit * p.rows + row0;
-          for (int j = 0; j < 9; ++j) tma_load_2d(sQ + j * 8192, &tm_q, &c->q_full, 64 * j, qy);
-          ++q_issued;
-          const int req = unit_req(p, pc.unit);
-          const int npg = (p.seqlens[req] + kPage - 1) / kPage;
-          const int pend = piece_page_end(pc, npg);
-          for (int pj = 2 * pc.t0; pj < pend; ++pj) {
-            const int slot = gp & 1;
-            if (!timed_wait(c, &c->page_empty[slot], ((gp >> 1) & 1) ^ 1, p)) { stop = true; break; }
-            const int pg = page_of(p, req, pj, npg);
-            mbar_arrive_expect_tx(&c->raw_full[slot], kRawB);
-            bulk_load(sS + slot * kSlotB + kRawOff, p.kcache_fp8 + (size_t)pg * kRawB, kRawB, &c->raw_full[slot]);
-            ++gp;
+      if (lane == 0 && !timed_wait(c, &c->q_empty, (pi & 1) ^ 1, p)) stop = true;
+      stop = __shfl_sync(0xffffffffu, stop ? 1 : 0, 0) != 0;
+      if (stop) break;
+      if (MODE == kModeNvfp4) {
+        // the warp dequantises the query rows: lane l converts values
+        // 16l..16l+15 of each row into slice l/4, chunks 2(l%4) and 2(l%4)+1;
+        // rows past this CTA's rows are zero
+        const size_t qrow0 = (size_t)pc.unit * p.rows + row0;
+        uint8_t* box = sQ + (lane >> 2) * 8192;
+#pragma unroll 1
+        for (int r0 = 0; r0 < kRowsPerCta; r0 += 8) {
+          uint2 cw[8];
+          uint32_t sb[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const bool live = r0 + i < rows_here;
+            const size_t qr = qrow0 + (live ? r0 + i : 0);
+            cw[i] = live ? *reinterpret_cast<const uint2*>(p.q_nvfp4 + qr * kNvfp4RowBytes + 8 * lane) : make_uint2(0, 0);
+            sb[i] = live ? p.q_scale[qr * kNvfp4ScaleBytes + lane] : 0u;
           }
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            uint4 lo, hi;
+            dequant_nvfp4_16(cw[i], sb[i], lo, hi);
+            *reinterpret_cast<uint4*>(sw128(box, r0 + i, 2 * (lane & 3))) = lo;
+            *reinterpret_cast<uint4*>(sw128(box, r0 + i, 2 * (lane & 3) + 1)) = hi;
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&c->q_full);
+      } else if (lane == 0) {
+        mbar_arrive_expect_tx(&c->q_full, kSl * 8192);
+        const int qy = pc.unit * p.rows + row0;
+        for (int j = 0; j < kSl; ++j) tma_load_2d(sQ + j * 8192, &tm_q, &c->q_full, 64 * j, qy);
+        ++q_issued;
+      }
+      if (lane == 0) {
+        const int req = unit_req(p, pc.unit);
+        const int npg = (p.seqlens[req] + kPage - 1) / kPage;
+        const int pend = piece_page_end(pc, npg);
+        for (int pj = 2 * pc.t0; pj < pend; ++pj) {
+          const int slot = gp & 1;
+          if (!timed_wait(c, &c->page_empty[slot], ((gp >> 1) & 1) ^ 1, p)) { stop = true; break; }
+          const size_t pg = (size_t)page_of(p, req, pj, npg);
+          uint8_t* dst = sS + slot * kSlotB + kRawOff;
+          mbar_arrive_expect_tx(&c->raw_full[slot], kRawB);
+          if (MODE == kModeNvfp4) {  // codes, then scales
+            bulk_load(dst, p.kcache_fp8 + pg * (kPage * kNvfp4RowBytes), kPage * kNvfp4RowBytes, &c->raw_full[slot]);
+            bulk_load(dst + kPage * kNvfp4RowBytes, p.kv_scale + pg * (kPage * kNvfp4ScaleBytes),
+                      kPage * kNvfp4ScaleBytes, &c->raw_full[slot]);
+          } else {
+            bulk_load(dst, p.kcache_fp8 + pg * kRawB, kRawB, &c->raw_full[slot]);
+          }
+          ++gp;
         }
       }
       stop = __shfl_sync(0xffffffffu, stop ? 1 : 0, 0) != 0;
@@ -181,7 +230,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp >= 8) {
     // ------------------------------------------------------------ converters
     const int tk = 8 * (warp - 8) + (lane & 7);  // token row of the page
-    const int qq = lane >> 3;                    // codes 128qq..128qq+127, RoPE chunks 2qq, 2qq+1
+    const int qq = lane >> 3;                    // latent values 128qq..128qq+127 (FP8: + RoPE chunks 2qq, 2qq+1)
     uint32_t cph = 0;
     int gp = 0;
     bool stop = false;
@@ -194,32 +243,64 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int slot = gp & 1;
         uint8_t* s = sS + slot * kSlotB;
         if (!timed_wait(c, &c->raw_full[slot], (gp >> 1) & 1, p)) { stop = true; break; }
-        // read this thread's 164 record bytes (8 lanes on 8 tokens per
-        // 16-byte access: the 656-byte stride puts them on distinct banks) ...
-        const uint8_t* rec = s + kRawOff + tk * kFp8RecordBytes;
-        uint4 cw[8], rope[2];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) cw[i] = *reinterpret_cast<const uint4*>(rec + 128 * qq + 16 * i);
-        const float sc = reinterpret_cast<const float*>(rec + 512)[qq];
-        rope[0] = *reinterpret_cast<const uint4*>(rec + 528 + 32 * qq);
-        rope[1] = *reinterpret_cast<const uint4*>(rec + 528 + 32 * qq + 16);
-        // ... and every converter's, before any slice row overwrites the records
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&c->grp_cv);
-        if (!timed_wait(c, &c->grp_cv, cph & 1, p)) { stop = true; break; }
-        ++cph;
+        // every converter reads its raw bytes before any slice row
+        // overwrites them (the slices overlap the raw area)
         const bool live = kPage * pj + tk < Ls;  // rows past the request's end are written as zeros
         const uint4 z = make_uint4(0, 0, 0, 0);
+        if (MODE == kModeNvfp4) {
+          // 64 code bytes (4 x 16) and 8 scale bytes; the 16-byte chunks are
+          // read in an order rotated by the token (the 256-byte row pitch
+          // would put 8 tokens on one bank group)
+          const uint8_t* codes = s + kRawOff + tk * kNvfp4RowBytes + 64 * qq;
+          uint4 cw[4];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          uint8_t* slice = s + (2 * qq + (i >> 2)) * 8192;
-          uint4 lo, hi;
-          dequant16(cw[i], sc, lo, hi);
-          *reinterpret_cast<uint4*>(sw128(slice, tk, 2 * (i & 3))) = live ? lo : z;
-          *reinterpret_cast<uint4*>(sw128(slice, tk, 2 * (i & 3) + 1)) = live ? hi : z;
+          for (int i = 0; i < 4; ++i) cw[i] = *reinterpret_cast<const uint4*>(codes + 16 * ((i + tk) & 3));
+          const uint2 scw = *reinterpret_cast<const uint2*>(s + kRawOff + kPage * kNvfp4RowBytes +
+                                                            tk * kNvfp4ScaleBytes + 8 * qq);
+          const unsigned long long sc8 = ((unsigned long long)scw.y << 32) | scw.x;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&c->grp_cv);
+          if (!timed_wait(c, &c->grp_cv, cph & 1, p)) { stop = true; break; }
+          ++cph;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            // chunk ch: values 128qq + 32ch .. +31 -> slice 2qq + ch/2, 16-B chunks 4(ch%2) .. 4(ch%2)+3
+            const int ch = (i + tk) & 3;
+            uint8_t* slice = s + (2 * qq + (ch >> 1)) * 8192;
+            const uint32_t sb = (uint32_t)(sc8 >> (16 * ch));
+            uint4 lo, hi;
+            dequant_nvfp4_16(make_uint2(cw[i].x, cw[i].y), sb & 0xFFu, lo, hi);
+            *reinterpret_cast<uint4*>(sw128(slice, tk, 4 * (ch & 1))) = live ? lo : z;
+            *reinterpret_cast<uint4*>(sw128(slice, tk, 4 * (ch & 1) + 1)) = live ? hi : z;
+            dequant_nvfp4_16(make_uint2(cw[i].z, cw[i].w), (sb >> 8) & 0xFFu, lo, hi);
+            *reinterpret_cast<uint4*>(sw128(slice, tk, 4 * (ch & 1) + 2)) = live ? lo : z;
+            *reinterpret_cast<uint4*>(sw128(slice, tk, 4 * (ch & 1) + 3)) = live ? hi : z;
+          }
+        } else {
+          // 164 record bytes (8 lanes on 8 tokens per 16-byte access: the
+          // 656-byte stride puts them on distinct banks)
+          const uint8_t* rec = s + kRawOff + tk * kFp8RecordBytes;
+          uint4 cw[8], rope[2];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) cw[i] = *reinterpret_cast<const uint4*>(rec + 128 * qq + 16 * i);
+          const float sc = reinterpret_cast<const float*>(rec + 512)[qq];
+          rope[0] = *reinterpret_cast<const uint4*>(rec + 528 + 32 * qq);
+          rope[1] = *reinterpret_cast<const uint4*>(rec + 528 + 32 * qq + 16);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&c->grp_cv);
+          if (!timed_wait(c, &c->grp_cv, cph & 1, p)) { stop = true; break; }
+          ++cph;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            uint8_t* slice = s + (2 * qq + (i >> 2)) * 8192;
+            uint4 lo, hi;
+            dequant16(cw[i], sc, lo, hi);
+            *reinterpret_cast<uint4*>(sw128(slice, tk, 2 * (i & 3))) = live ? lo : z;
+            *reinterpret_cast<uint4*>(sw128(slice, tk, 2 * (i & 3) + 1)) = live ? hi : z;
+          }
+          *reinterpret_cast<uint4*>(sw128(s + 8 * 8192, tk, 2 * qq)) = live ? rope[0] : z;
+          *reinterpret_cast<uint4*>(sw128(s + 8 * 8192, tk, 2 * qq + 1)) = live ? rope[1] : z;
         }
-        *reinterpret_cast<uint4*>(sw128(s + 8 * 8192, tk, 2 * qq)) = live ? rope[0] : z;
-        *reinterpret_cast<uint4*>(sw128(s + 8 * 8192, tk, 2 * qq + 1)) = live ? rope[1] : z;
         fence_proxy_async_smem();  // this thread's slice rows -> the tensor core
         __syncwarp();
         if (lane == 0) mbar_arrive(&c->page_full[slot]);
@@ -245,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             const uint32_t d = tmem + kTmemS + 64 * b;
             const uint32_t qa = smem_u32(sQ), kb = smem_u32(sS + b * kSlotB);
-            for (int j = 0; j < 9; ++j) {
+            for (int j = 0; j < kSl; ++j) {
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk)
                 mma_bf16_ss(d, sdesc(qa + j * 8192 + kk * 32, 16, 1024), sdesc(kb + j * 8192 + kk * 32, 16, 1024),
@@ -478,26 +559,33 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) tmem_dealloc(tmem, kTmemCols);
 }
 
-template <int NR>
-cudaError_t launch_fp8(const CUtensorMap& tq, const DecodeParams& p, int parts, int row_groups,
-                       cudaStream_t stream) {
+template <int NR, int MODE>
+cudaError_t launch_page(const CUtensorMap& tq, const DecodeParams& p, int parts, int row_groups,
+                        cudaStream_t stream) {
   constexpr int smem = Smem<NR>::total + 1024;
-  auto kern = mla_decode_fp8_kernel<NR>;
+  auto kern = mla_decode_page_kernel<NR, MODE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   e = launch_pdl(kern, dim3(parts, row_groups), dim3(kThreads), smem, stream, tq, p);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
-}  // namespace
-
-cudaError_t launch_decode_fp8(int rows_per_cta, const CUtensorMap& tq, const DecodeParams& p, int parts,
-                              int row_groups, cudaStream_t stream) {
+template <int MODE>
+cudaError_t launch_rows(int rows_per_cta, const CUtensorMap& tq, const DecodeParams& p, int parts, int row_groups,
+                        cudaStream_t stream) {
   // <= 16 rows run in the 32-row kernel: the extra P^T rows are written as
   // zeros and their output rows are never stored
-  if (rows_per_cta <= 32) return launch_fp8<32>(tq, p, parts, row_groups, stream);
-  if (rows_per_cta <= 48) return launch_fp8<48>(tq, p, parts, row_groups, stream);
-  return launch_fp8<64>(tq, p, parts, row_groups, stream);
+  if (rows_per_cta <= 32) return launch_page<32, MODE>(tq, p, parts, row_groups, stream);
+  if (rows_per_cta <= 48) return launch_page<48, MODE>(tq, p, parts, row_groups, stream);
+  return launch_page<64, MODE>(tq, p, parts, row_groups, stream);
+}
+
+}  // namespace
+
+cudaError_t launch_decode_page(int mode, int rows_per_cta, const CUtensorMap& tq, const DecodeParams& p, int parts,
+                               int row_groups, cudaStream_t stream) {
+  if (mode == kModeNvfp4) return launch_rows<kModeNvfp4>(rows_per_cta, tq, p, parts, row_groups, stream);
+  return launch_rows<kModeFp8>(rows_per_cta, tq, p, parts, row_groups, stream);
 }
 
 }  // namespace mla

@@ -84,19 +84,20 @@ cudaError_t launch_pdl(void (*kern)(Params...), dim3 grid, dim3 block, size_t sm
 cudaError_t launch_decode(int rows_per_cta, int mode, const CUtensorMap& tq, const CUtensorMap& tkv,
                           const CUtensorMap& tv, const DecodeParams& p, int parts, int row_groups,
                           cudaStream_t stream);
-// FP8 paged cache: each page fetched by one bulk copy and converted once
-// (no cache tensor map).
-cudaError_t launch_decode_fp8(int rows_per_cta, const CUtensorMap& tq, const DecodeParams& p, int parts,
-                              int row_groups, cudaStream_t stream);
+// FP8 or NVFP4 paged cache (mode kModeFp8 / kModeNvfp4): each page fetched by
+// bulk copies and converted once (no cache tensor map; NVFP4 needs no tq).
+cudaError_t launch_decode_page(int mode, int rows_per_cta, const CUtensorMap& tq, const DecodeParams& p, int parts,
+                               int row_groups, cudaStream_t stream);
 // Units of more than 64 rows, BF16 cache (paged, or token-sparse when `sparse`):
 // CTA pairs (clusters of two), one per part.
 cudaError_t launch_decode_pair(const CUtensorMap& tq, const CUtensorMap& tkv, const CUtensorMap& tv,
                                const DecodeParams& p, int parts, bool sparse, cudaStream_t stream);
 // How many CTA pairs of the pair kernel can be resident at once on the current device (0 if unknown).
 int max_pair_clusters();
-// Unit u reads seqlens[u / upr] (paged decoding; upr = units per request).
-mla_status_t launch_metadata(const int32_t* seqlens, int U, int upr, int topk, int parts, int32_t* tile_md,
-                             int32_t* num_splits, cudaStream_t stream);
+// Unit u reads seqlens[u / upr] (paged decoding; upr = units per request);
+// rows = query rows per unit.
+mla_status_t launch_metadata(const int32_t* seqlens, int U, int upr, int topk, int parts, int rows,
+                             int32_t* tile_md, int32_t* num_splits, cudaStream_t stream);
 // `sink` (device fp32 [h_q] or null): the head of row r of a unit is r % h_q.
 mla_status_t launch_combine(const void* workspace, int units, int rows, int parts, const int32_t* split_ptr,
                             int h_q, const float* sink, void* out, float* lse, cudaStream_t stream);

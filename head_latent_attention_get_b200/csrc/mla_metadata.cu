@@ -57,6 +57,35 @@ __host__ __device__ inline int first_part_of(int Cu, int payload) {
   return (int)((Cu + kSchedOverhead) / payload);
 }
 
+// Equal units of more than 64 rows. Their kernels (the CTA pair, or two
+// row-group CTAs) run the keys in steps of two tiles, and every piece pays a
+// pipeline fill and a partial-result write. When every unit has the same n
+// tiles and there are at least two parts per unit, the cost-axis cut would
+// hand some parts a run that ends half a step into a unit plus a second
+// piece; instead each unit is cut into k = min(parts / units, ceil(n / 2))
+// pieces of whole steps (as equal as steps allow), one piece per part, and
+// the parts past k * units get no work. Returns k, or 0 when the cost-axis
+// plan applies.
+__host__ __device__ inline int equal_unit_pieces(int U, int parts, int rows, int n_min, int n_max) {
+  if (rows <= 64 || U <= 0 || n_min != n_max || n_min <= 0) return 0;
+  const int k = min(parts / U, (n_min + 1) / 2);
+  return k >= 2 ? k : 0;
+}
+// Part p of the equal-unit plan: piece p % k of unit p / k, tiles
+// [2 floor(j s / k), min(2 floor((j+1) s / k), n)) with s = ceil(n / 2) steps.
+__host__ __device__ inline void equal_unit_part(int p, int U, int k, int n, int32_t* md) {
+  const int steps = (n + 1) / 2;
+  if (p >= U * k) {
+    md[0] = U; md[1] = 0; md[2] = U; md[3] = 0; md[4] = 0;
+  } else {
+    const int u = p / k, j = p - u * k;
+    md[0] = u; md[1] = 2 * (int)((long long)j * steps / k);
+    md[2] = u; md[3] = min(n, 2 * (int)((long long)(j + 1) * steps / k));
+    md[4] = p;  // the unit's splits are u*k .. u*k + k-1
+  }
+  md[5] = k; md[6] = 0; md[7] = 0;
+}
+
 // ---------------------------------------------------------------- host twin
 extern "C" mla_status_t mla_get_metadata_host(const int32_t* cache_seqlens, int batch, int s_q, int h_q,
                                               int h_kv, int topk, int num_sm_parts, int32_t* tile_md,
@@ -69,6 +98,18 @@ extern "C" mla_status_t mla_get_metadata_host(const int32_t* cache_seqlens, int 
   Geometry g;
   if (!unit_geometry(s_q, h_q, h_kv, topk, &g)) return MLA_ERR_UNSUPPORTED;
   const int U = batch * g.units_per_req;
+  int n_min = 0x7fffffff, n_max = 0;
+  for (int u = 0; u < U; ++u) {
+    const int n = unit_tiles(cache_seqlens, u, g.units_per_req, topk);
+    n_min = n < n_min ? n : n_min;
+    n_max = n > n_max ? n : n_max;
+  }
+  const int k = equal_unit_pieces(U, num_sm_parts, g.rows, n_min, n_max);
+  if (k > 0) {
+    for (int p = 0; p < num_sm_parts; ++p) equal_unit_part(p, U, k, n_max, tile_md + p * MLA_TILE_MD_INTS);
+    for (int u = 0; u <= U; ++u) num_splits[u] = u * k;
+    return MLA_OK;
+  }
   // cost prefix C[0..U] kept in num_splits first, then replaced by split pointers
   int total = 0, max_cost = 0;
   for (int u = 0; u < U; ++u) {
@@ -143,15 +184,34 @@ __device__ int block_max(int v) {
   for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
   if (lane == 0) warp_max[warp] = v;
   __syncthreads();
-  int m = 0;
+  int m = warp_max[0];
 #pragma unroll
-  for (int i = 0; i < kMetaThreads / 32; ++i) m = max(m, warp_max[i]);
+  for (int i = 1; i < kMetaThreads / 32; ++i) m = max(m, warp_max[i]);
   __syncthreads();
   return m;
 }
 
+// Equal-unit plan on the device (every thread of the block takes the same
+// branch: n_min and n_max are block-wide). Returns true if it wrote the plan.
+__device__ bool equal_unit_plan(const int32_t* seqlens, int U, int upr, int topk, int parts, int rows, int u0, int u1,
+                                int32_t* tile_md, int32_t* num_splits) {
+  int lo = 0x7fffffff, hi = 0;
+  for (int u = u0; u < u1; ++u) {
+    const int n = unit_tiles(seqlens, u, upr, topk);
+    lo = min(lo, n);
+    hi = max(hi, n);
+  }
+  const int n_max = block_max(hi);
+  const int n_min = -block_max(-lo);
+  const int k = equal_unit_pieces(U, parts, rows, n_min, n_max);
+  if (k == 0) return false;
+  for (int p = threadIdx.x; p < parts; p += kMetaThreads) equal_unit_part(p, U, k, n_max, tile_md + p * MLA_TILE_MD_INTS);
+  for (int u = threadIdx.x; u <= U; u += kMetaThreads) num_splits[u] = u * k;
+  return true;
+}
+
 __global__ void __launch_bounds__(kMetaThreads) mla_metadata_kernel(const int32_t* __restrict__ seqlens,
-                                                                   int U, int upr, int topk, int parts,
+                                                                   int U, int upr, int topk, int parts, int rows,
                                                                    int32_t* __restrict__ tile_md,
                                                                    int32_t* __restrict__ num_splits) {
   griddep_launch_dependents();  // the decode kernel may start its set-up (it waits for this grid)
@@ -159,6 +219,7 @@ __global__ void __launch_bounds__(kMetaThreads) mla_metadata_kernel(const int32_
   const int t = threadIdx.x;
   const int per = (U + kMetaThreads - 1) / kMetaThreads;
   const int u0 = min(U, t * per), u1 = min(U, u0 + per);
+  if (equal_unit_plan(seqlens, U, upr, topk, parts, rows, u0, u1, tile_md, num_splits)) return;
   // 1. cost prefix C[u] -> num_splits[u], total -> num_splits[U]
   int my = 0, my_max = 0;
   for (int u = u0; u < u1; ++u) {
@@ -227,7 +288,7 @@ __global__ void __launch_bounds__(kMetaThreads) mla_metadata_kernel(const int32_
 constexpr int kMetaSmemUnits = 4096;
 
 __global__ void __launch_bounds__(kMetaThreads) mla_metadata_smem_kernel(const int32_t* __restrict__ seqlens,
-                                                                        int U, int upr, int topk, int parts,
+                                                                        int U, int upr, int topk, int parts, int rows,
                                                                         int32_t* __restrict__ tile_md,
                                                                         int32_t* __restrict__ num_splits) {
   griddep_launch_dependents();  // the decode kernel may start its set-up (it waits for this grid)
@@ -237,6 +298,7 @@ __global__ void __launch_bounds__(kMetaThreads) mla_metadata_smem_kernel(const i
   const int t = threadIdx.x;
   const int per = (U + kMetaThreads - 1) / kMetaThreads;
   const int u0 = min(U, t * per), u1 = min(U, u0 + per);
+  if (equal_unit_plan(seqlens, U, upr, topk, parts, rows, u0, u1, tile_md, num_splits)) return;
   // 1. cost prefix C[0..U]
   int my = 0, my_max = 0;
   for (int u = u0; u < u1; ++u) {
@@ -292,12 +354,12 @@ __global__ void __launch_bounds__(kMetaThreads) mla_metadata_smem_kernel(const i
   }
 }
 
-mla_status_t launch_metadata(const int32_t* seqlens, int U, int upr, int topk, int parts, int32_t* tile_md,
-                             int32_t* num_splits, cudaStream_t stream) {
+mla_status_t launch_metadata(const int32_t* seqlens, int U, int upr, int topk, int parts, int rows,
+                             int32_t* tile_md, int32_t* num_splits, cudaStream_t stream) {
   if (U <= kMetaSmemUnits)
-    mla_metadata_smem_kernel<<<1, kMetaThreads, 0, stream>>>(seqlens, U, upr, topk, parts, tile_md, num_splits);
+    mla_metadata_smem_kernel<<<1, kMetaThreads, 0, stream>>>(seqlens, U, upr, topk, parts, rows, tile_md, num_splits);
   else
-    mla_metadata_kernel<<<1, kMetaThreads, 0, stream>>>(seqlens, U, upr, topk, parts, tile_md, num_splits);
+    mla_metadata_kernel<<<1, kMetaThreads, 0, stream>>>(seqlens, U, upr, topk, parts, rows, tile_md, num_splits);
   return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 

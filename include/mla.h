@@ -152,6 +152,12 @@ mla_status_t mla_get_num_sm_parts(int device, int s_q, int h_q, int h_kv, int to
  * ceil(total / num_sm_parts), raised to the largest unit's cost when that is
  * at most 8 blocks more (equal units then take one part each and are not
  * split; the trailing parts get no work). The total cost must stay below 2^31.
+ * One exception: when every unit has the same n > 0 blocks, a unit holds
+ * more than 64 query rows, and num_sm_parts >= 2 * units, each unit is cut
+ * into k = min(num_sm_parts / units, ceil(n / 2)) pieces of whole pairs of
+ * blocks (their lengths differ by at most one pair), piece j of unit u goes
+ * to part u*k + j, and the parts past k * units get no work (their range
+ * begins and ends at {units, 0}). Cost per part is then reported as k.
  *
  *   cache_seqlens  device int32 [batch]; read only when topk == 0 (may be
  *                  NULL when topk > 0).

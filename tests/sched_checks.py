@@ -4,7 +4,9 @@ Any exact cover is a valid schedule, so these checks test properties, not
 bytes: every (unit, tile) pair lands in exactly one part, parts are
 contiguous, the split counts match the parts that touch each unit, each
 piece's workspace slot is unique within its unit, and no part carries much
-more than its share of the cost.
+more than its share of the cost (or, for equal units of more than 64 rows
+with two or more parts per unit, every unit is cut into equal pieces of
+whole 2-tile steps).
 """
 import numpy as np
 
@@ -36,6 +38,7 @@ def unit_tiles(seqlens, batch, s_q, topk, h_q=None):
 
 
 def pieces_of_part(md, n):
+    """(unit, first tile, end tile, first piece of the part) of each piece."""
     bu, bt, eu, et, first_ws = (int(x) for x in md[:5])
     out = []
     u, t, first = bu, bt, True
@@ -49,8 +52,30 @@ def pieces_of_part(md, n):
     return out
 
 
+def rows_per_unit(s_q, h_q, topk):
+    """Query rows of one unit; None when h_q is not given."""
+    if h_q is None:
+        return None
+    if topk:
+        return h_q
+    return s_q * h_q // units_per_request(s_q, h_q, topk)
+
+
+def equal_unit_pieces(n, parts, rows):
+    """Pieces per unit of the equal-unit plan (units of more than 64 rows,
+    all with the same tile count n0 > 0, at least two parts per unit):
+    k = min(parts // units, ceil(n0 / 2)), or 0 when the cost-axis plan
+    applies."""
+    U = len(n)
+    if rows is None or rows <= 64 or U == 0 or min(n) != max(n) or n[0] <= 0:
+        return 0
+    k = min(parts // U, (n[0] + 1) // 2)
+    return k if k >= 2 else 0
+
+
 def check_schedule(tile_md, num_splits, seqlens, batch, s_q, topk, parts, h_q=None):
-    """h_q=None: one unit per request (s_q*h_q <= 128) on the paged path."""
+    """h_q=None: one unit per request (s_q*h_q <= 128) on the paged path, with
+    at most 64 rows."""
     n = unit_tiles(seqlens, batch, s_q, topk, h_q)
     U = len(n)
     md = np.asarray(tile_md).reshape(parts, 8)
@@ -82,6 +107,21 @@ def check_schedule(tile_md, num_splits, seqlens, batch, s_q, topk, parts, h_q=No
                 ws = int(md[p][4]) if first else int(ptr[u])
                 assert ws == ptr[u] + j, (u, p, ws, ptr[u] + j)
     assert ptr[U] <= U + parts
+    k = equal_unit_pieces(n, parts, rows_per_unit(s_q, h_q, topk))
+    if k:
+        # every unit cut into k pieces of whole 2-tile steps, one per part:
+        # piece lengths differ by at most one step, later parts are empty
+        steps = (n[0] + 1) // 2
+        assert list(ptr) == [u * k for u in range(U + 1)]
+        for p in range(parts):
+            pcs = pieces_of_part(md[p], n)
+            if p >= U * k:
+                assert pcs == []
+                continue
+            (u, t0, t1, _), = pcs
+            assert u == p // k and t0 % 2 == 0
+            assert -(-(t1 - t0) // 2) in (steps // k, -(-steps // k))
+        return {"payload": None, "max_cost": max(cost), "splits": int(ptr[U]), "equal_pieces": k}
     total = sum(x + OVERHEAD for x in n if x > 0)
     even = -(-total // parts) if total else 1
     unit_max = max([x + OVERHEAD for x in n if x > 0], default=0)

@@ -155,6 +155,10 @@ def host_schedule(seqlens, batch, s_q, h_q, topk, parts):
     ("mtp6_64heads", [4096, 300, 0, 9000], 6, 64, 0, 74),
     ("rows96_blocks", [70, 129, 5000], 3, 64, 0, 74),
     ("256heads", [4096] * 8, 1, 256, 0, 74),
+    ("equal_units_two_pieces", [32768] * 32, 1, 128, 2048, 74),
+    ("equal_units_odd_steps", [300] * 7, 1, 100, 0, 40),
+    ("equal_units_more_parts_than_steps", [200] * 3, 1, 128, 0, 148),
+    ("equal_units_64_rows_cost_axis", [32768] * 32, 1, 64, 2048, 148),
 ])
 def test_host_scheduler_invariants(case):
     _, lens, s_q, h_q, topk, parts = case

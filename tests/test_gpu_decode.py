@@ -20,14 +20,16 @@ def _dense(name="tiny", **over):
 
 
 # ------------------------------------------------------------------ scheduler
-@pytest.mark.parametrize("lens,s_q,h_q,topk", [
-    ([70, 129], 1, 16, 0), ([4096] * 64, 1, 128, 0), ([0, 5, 0, 300, 9000], 2, 16, 0),
-    (list(range(0, 30000, 97)), 1, 64, 0), ([32768] * 32, 1, 128, 2048), ([100] * 5, 2, 32, 128),
-    ([(37 * i) % 5000 for i in range(13000)], 1, 16, 0),      # more units than the shared-memory prefix holds
-    ([4096] * 64, 6, 64, 0)])                                 # three row-block units per request
-def test_metadata_device_matches_host_twin(lens, s_q, h_q, topk):
+@pytest.mark.parametrize("lens,s_q,h_q,topk,parts", [
+    ([70, 129], 1, 16, 0, None), ([4096] * 64, 1, 128, 0, None), ([0, 5, 0, 300, 9000], 2, 16, 0, None),
+    (list(range(0, 30000, 97)), 1, 64, 0, None), ([32768] * 32, 1, 128, 2048, None),   # equal units, 2 pieces each
+    ([100] * 5, 2, 32, 128, None),
+    ([(37 * i) % 5000 for i in range(13000)], 1, 16, 0, None),  # more units than the shared-memory prefix holds
+    ([3000] * 5000, 1, 128, 0, 10003),                          # the same, equal units, 2 pieces each
+    ([4096] * 64, 6, 64, 0, None)])                             # three row-block units per request
+def test_metadata_device_matches_host_twin(lens, s_q, h_q, topk, parts):
     B = len(lens)
-    parts = M.mla_get_num_sm_parts(0, s_q, h_q, 1, topk)
+    parts = parts or M.mla_get_num_sm_parts(0, s_q, h_q, 1, topk)
     U = B * M.mla_decode_geometry(s_q, h_q, 1, topk)[0]
     md_h = np.zeros(parts * 8, np.int32)
     ns_h = np.zeros(U + 1, np.int32)
