@@ -197,3 +197,21 @@ def test_combine_strides_over_more_items_than_blocks():
     assert (np.diff(ns) > 1).sum() > 50            # many units are split
     G.compare_full(inp, out, lse, "400 requests, 6400 combine items")
     assert r.status()[0] == C.MLA_OK
+
+
+@pytest.mark.parametrize("kv", ["bf16", "fp8"])
+def test_repeated_calls_on_one_workspace_are_identical(kv):
+    """Five calls on one workspace, with split requests and empty ones among
+    them, give the same bits each time (nothing a call leaves in the
+    workspace changes the next)."""
+    w = _dense(batch=5, seqlens=[3000, 0, 129, 5000, 0], h_q=64, seed=808, kv=kv)
+    inp = W.make_inputs(w, poison_tail=True)
+    out, lse, r = G.run_gpu(inp, runner_kwargs={"num_sm_parts": 7})
+    assert (np.diff(r.num_splits.cpu().numpy()) > 1).any()
+    G.compare_full(inp, out, lse, f"{kv} first call")
+    for _ in range(4):
+        o2, l2 = r.run()
+        torch.cuda.synchronize()
+        assert torch.equal(o2.float().cpu(), torch.from_numpy(out))
+        assert np.array_equal(l2.cpu().numpy().view(np.uint32), lse.view(np.uint32))
+    assert r.status()[0] == C.MLA_OK
