@@ -265,6 +265,7 @@ mla_status_t mla_combine_sink(const void* workspace, size_t workspace_bytes, con
   if (!aligned16(out) || !aligned16(workspace)) return MLA_ERR_INVALID_ARG;
   if (sink && (h_q <= 0 || (reinterpret_cast<uintptr_t>(sink) & 3u) != 0))
     return MLA_ERR_INVALID_ARG;
+  if ((long long)num_units * rows_per_unit > 0x7fffffffLL / kDqk) return MLA_ERR_UNSUPPORTED;
   if (workspace_bytes < ws_layout(num_units, rows_per_unit, num_sm_parts).total)
     return MLA_ERR_WORKSPACE_TOO_SMALL;
   return launch_combine(workspace, num_units, rows_per_unit, num_sm_parts, num_splits, sink ? h_q : 1, sink, out,

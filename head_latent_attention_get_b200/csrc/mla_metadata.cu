@@ -215,6 +215,7 @@ __global__ void __launch_bounds__(kMetaThreads) mla_metadata_kernel(const int32_
                                                                    int32_t* __restrict__ tile_md,
                                                                    int32_t* __restrict__ num_splits) {
   griddep_launch_dependents();  // the decode kernel may start its set-up (it waits for this grid)
+  griddep_wait();  // launched early behind the previous kernel: its reads of tile_md / num_splits are done
   __shared__ int s_payload;
   const int t = threadIdx.x;
   const int per = (U + kMetaThreads - 1) / kMetaThreads;
@@ -292,6 +293,7 @@ __global__ void __launch_bounds__(kMetaThreads) mla_metadata_smem_kernel(const i
                                                                         int32_t* __restrict__ tile_md,
                                                                         int32_t* __restrict__ num_splits) {
   griddep_launch_dependents();  // the decode kernel may start its set-up (it waits for this grid)
+  griddep_wait();  // launched early behind the previous kernel: its reads of tile_md / num_splits are done
   __shared__ int32_t C[kMetaSmemUnits + 1];  // cost prefix
   __shared__ int32_t S[kMetaSmemUnits + 1];  // split prefix
   __shared__ int s_payload;
@@ -356,11 +358,16 @@ __global__ void __launch_bounds__(kMetaThreads) mla_metadata_smem_kernel(const i
 
 mla_status_t launch_metadata(const int32_t* seqlens, int U, int upr, int topk, int parts, int rows,
                              int32_t* tile_md, int32_t* num_splits, cudaStream_t stream) {
-  if (U <= kMetaSmemUnits)
-    mla_metadata_smem_kernel<<<1, kMetaThreads, 0, stream>>>(seqlens, U, upr, topk, parts, rows, tile_md, num_splits);
-  else
-    mla_metadata_kernel<<<1, kMetaThreads, 0, stream>>>(seqlens, U, upr, topk, parts, rows, tile_md, num_splits);
-  return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+  // programmatic dependent launch: the block is scheduled while the previous
+  // kernel of the stream (e.g. the last step's combine) finishes, and waits
+  // for it before reading or writing anything
+  const cudaError_t e =
+      U <= kMetaSmemUnits
+          ? launch_pdl(mla_metadata_smem_kernel, dim3(1), dim3(kMetaThreads), 0, stream, seqlens, U, upr, topk, parts,
+                       rows, tile_md, num_splits)
+          : launch_pdl(mla_metadata_kernel, dim3(1), dim3(kMetaThreads), 0, stream, seqlens, U, upr, topk, parts, rows,
+                       tile_md, num_splits);
+  return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? MLA_OK : MLA_ERR_CUDA;
 }
 
 }  // namespace mla
