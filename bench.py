@@ -46,11 +46,18 @@ def load_peaks():
     return dict(PEAK_FALLBACK), "fallback"
 
 
-def kernel_source_hash() -> str:
+KERNEL_SOURCE = {"mla_decode_pair_kernel": "mla_decode_pair.cu", "mla_decode_kernel": "mla_decode.cu",
+                 "mla_decode_page_kernel": "mla_decode_page.cu"}
+
+
+def kernel_source_hash(kernel: str) -> str:
+    """Hash of what one decode kernel is built from: its own .cu file and the
+    shared headers (the scheduler, combine and host-side files do not change
+    the kernel's memory traffic)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "head_latent_attention_get_b200", "csrc")
     for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh")):
+        if f.endswith(".cuh") or f == KERNEL_SOURCE[kernel]:
             with open(os.path.join(csrc, f), "rb") as fh:
                 h.update(fh.read())
     return h.hexdigest()[:16]
@@ -76,7 +83,7 @@ def recorded_traffic(workload: str):
     with open(p) as f:
         d = json.load(f)
     e = d.get(workload)
-    if not e or e.get("kernel_source_sha") != kernel_source_hash():
+    if not e or e.get("kernel") not in KERNEL_SOURCE or e.get("kernel_source_sha") != kernel_source_hash(e["kernel"]):
         return None
     return e.get("dram_bytes_per_launch")
 
