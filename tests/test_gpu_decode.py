@@ -167,12 +167,13 @@ def test_bounds_status_without_fault():
     G.compare(out[1:], lse[1:], ref_o, ref_l, "unaffected request")
 
 
-@pytest.mark.parametrize("kv", ["bf16", "fp8"])
+@pytest.mark.parametrize("kv", ["bf16", "fp8", "nvfp4"])
 def test_timeout_status_and_context_survives(kv):
     """Scores withheld from the softmax: every bounded wait gives up, the
     status word says so and the next call on the same context is exact (the
-    bf16 row-group kernel and the FP8 page kernel)."""
-    inp = W.make_inputs(_dense("tiny", kv=kv))
+    bf16 row-group kernel and the page kernel with FP8 and NVFP4 pages)."""
+    over = {"scale": 512 ** -0.5} if kv == "nvfp4" else {}
+    inp = W.make_inputs(_dense("tiny", kv=kv, **over))
     _, _, r = G.run_gpu(inp, runner_kwargs={"timeout_ns": 20_000_000,
                                             "debug_flags": C.MLA_DEBUG_WITHHOLD_SCORES})
     code, bits = r.status()
