@@ -168,7 +168,8 @@ def workload_config(inp, work):
            "algorithmic_flops": work["flops"], "algorithmic_bytes": work["bytes"],
            "l2": ("a step reads %.0f MB (more than twice the 126 MB L2), no flush" if
                   work["bytes"] >= 2 * L2_BYTES else
-                  "a step reads %.0f MB (less than twice L2): 256 MB written before every step") % (
+                  "a step reads %.0f MB (less than twice L2): 256 MB written before every step, "
+                  "outside the events that time it") % (
                work["bytes"] / 1e6)}
     if w.topk:
         cfg["topk"] = w.topk
@@ -309,20 +310,23 @@ def measure(inp, steps: int, warmup: int, dev, pg=None):
     flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev) if touched < 2 * L2_BYTES else None
 
     def step(ev=None):
+        """ev: four events (one around each kernel) or two (around the whole
+        step, whose kernels then stay chained)."""
+        each = ev is not None and len(ev) == 4
         if flush is not None:
             flush.fill_(1)
         if ev is not None:
             ev[0].record(stream)
         runner.plan(stream)
-        if ev is not None:
+        if each:
             ev[1].record(stream)
         runner.run(stream)
-        if ev is not None:
+        if each:
             ev[2].record(stream)
         M.mla_combine_sink(runner.workspace, ws_bytes, runner.num_splits, U, R, P, w.h_q, d["sink"], runner.out,
                            runner.lse, stream)
         if ev is not None:
-            ev[3].record(stream)
+            ev[-1].record(stream)
 
     for _ in range(warmup):
         step()
@@ -331,6 +335,7 @@ def measure(inp, steps: int, warmup: int, dev, pg=None):
     if code != C.MLA_OK:
         raise RuntimeError(f"{w.name}: device status after warm-up: {M.mla_status_string(code)} bits={bits}")
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    whole = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     bad_reasons = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
@@ -341,11 +346,15 @@ def measure(inp, steps: int, warmup: int, dev, pg=None):
         torch.cuda.synchronize()
         with ClockSampler(dev) as clocks:
             # whole steps back to back (the kernels of a step overlap their
-            # launches), then the same steps with an event around each kernel
+            # launches), then the same steps with events around each whole
+            # step (the L2 flush stays outside them), then with an event
+            # around each kernel
             t_start.record(stream)
             for s in range(steps):
                 step()
             t_end.record(stream)
+            for s in range(steps):
+                step(whole[s])
             for s in range(steps):
                 step(evs[s])
             torch.cuda.synchronize()
@@ -361,6 +370,7 @@ def measure(inp, steps: int, warmup: int, dev, pg=None):
     return {"runner": runner, "rows": runner.rows, "dev_inputs": d, "total_ms": t_start.elapsed_time(t_end), "steps": steps,
             "flushed": flush is not None, "metadata_ms": sum(meta) / steps, "kernel_ms": sum(dec) / steps,
             "combine_ms": sum(comb) / steps, "step_kernels_ms": (sum(meta) + sum(dec) + sum(comb)) / steps,
+            "step_chained_ms": sum(e[0].elapsed_time(e[1]) for e in whole) / steps,
             "clocks": dict(clocks.summary(), remeasured=remeasured), "launches": 3 * steps}
 
 
@@ -409,7 +419,9 @@ def run_gpu(args):
     work = W.algorithmic_work(inp)
     w = inp.workload
     m = measure(inp, args.steps, args.warmup, dev, pg)
-    ms_step = max_over_ranks(pg, m["total_ms"] / args.steps, dev)
+    # with an L2 flush before every step, the step is timed between events
+    # around it (the flush outside); otherwise steps run back to back
+    ms_step = max_over_ranks(pg, m["step_chained_ms"] if m["flushed"] else m["total_ms"] / args.steps, dev)
     runner, d = m["runner"], m["dev_inputs"]
     stream = torch.cuda.current_stream()
 
@@ -496,8 +508,8 @@ def run_gpu(args):
             r = roofline_of(pi, pm, peaks, peak_src)
             r.update({"workload": W.get_workload(name).note, "steps": pm["steps"],
                       "l2_flush_between_steps": pm["flushed"], "clocks": pm["clocks"],
-                      # with an L2 flush in every step, the step time is the sum of its kernels
-                      "step_ms": pm["step_kernels_ms"] if pm["flushed"] else pm["total_ms"] / pm["steps"]})
+                      # with an L2 flush before every step: events around each whole step
+                      "step_ms": pm["step_chained_ms"] if pm["flushed"] else pm["total_ms"] / pm["steps"]})
             r["step_tflops"] = W.algorithmic_work(pi)["flops"] / (r["step_ms"] * 1e-3) / 1e12
             per_config[name] = r
             del pm
