@@ -387,6 +387,9 @@ def roofline_of(inp, m, peaks, peak_src):
     t_tc = work["flops"] / (tc_peak * 1e12)
     bound = "hbm" if t_hbm >= t_tc else "tensor"
     mhz = m["clocks"].get("sm_mhz")
+    # with an L2 flush before every step: events around each whole step;
+    # otherwise whole steps back to back
+    step_ms = m["step_chained_ms"] if m["flushed"] else m["total_ms"] / m["steps"]
     return {"bound": bound,
             "achieved": achieved_gbs if bound == "hbm" else achieved_tf,
             "peak": hbm_peak if bound == "hbm" else tc_peak,
@@ -401,7 +404,11 @@ def roofline_of(inp, m, peaks, peak_src):
             "achieved_tflops": achieved_tf, "achieved_gbs": achieved_gbs,
             "hbm_frac": achieved_gbs / hbm_peak, "tensor_frac": achieved_tf / tc_peak,
             "roofline_frac": max(t_hbm, t_tc) / (k_ms * 1e-3),
-            "combine_ms": m["combine_ms"], "metadata_ms": m["metadata_ms"]}
+            "combine_ms": m["combine_ms"], "metadata_ms": m["metadata_ms"],
+            "step_ms": step_ms, "step_overhead_ms": step_ms - k_ms,
+            "timing": "kernel_ms, metadata_ms, combine_ms: each kernel between its own events (its launch "
+                      "gap included); step_ms: scheduler, decode and combine chained by programmatic dependent "
+                      "launch; step_overhead_ms = step_ms - kernel_ms, what the scheduler and combine add"}
 
 
 def run_gpu(args):
@@ -507,9 +514,7 @@ def run_gpu(args):
             pm = measure(pi, min(args.steps, args.per_config_steps), args.warmup, dev, pg)
             r = roofline_of(pi, pm, peaks, peak_src)
             r.update({"workload": W.get_workload(name).note, "steps": pm["steps"],
-                      "l2_flush_between_steps": pm["flushed"], "clocks": pm["clocks"],
-                      # with an L2 flush before every step: events around each whole step
-                      "step_ms": pm["step_chained_ms"] if pm["flushed"] else pm["total_ms"] / pm["steps"]})
+                      "l2_flush_between_steps": pm["flushed"], "clocks": pm["clocks"]})
             r["step_tflops"] = W.algorithmic_work(pi)["flops"] / (r["step_ms"] * 1e-3) / 1e12
             per_config[name] = r
             del pm
