@@ -408,7 +408,9 @@ def roofline_of(inp, m, peaks, peak_src):
             "step_ms": step_ms, "step_overhead_ms": step_ms - k_ms,
             "timing": "kernel_ms, metadata_ms, combine_ms: each kernel between its own events (its launch "
                       "gap included); step_ms: scheduler, decode and combine chained by programmatic dependent "
-                      "launch; step_overhead_ms = step_ms - kernel_ms, what the scheduler and combine add"}
+                      "launch; step_overhead_ms = step_ms - kernel_ms, what the scheduler and combine add (the two come "
+                      "from separate passes: where the power cap moves the SM clock between them it can read "
+                      "below zero)"}
 
 
 def run_gpu(args):

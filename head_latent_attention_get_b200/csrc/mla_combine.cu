@@ -9,7 +9,8 @@
 // split at all gets out 0 and lse sigma.
 // One warp merges one output row: every lane walks the row's splits in order
 // (the lse values are broadcast loads) and owns 16 of the 512 dims, so each
-// split's partial row is read with coalesced 16-byte loads; a row whose unit
+// split's partial row is read with coalesced 16-byte loads (the first two
+// splits' rows are requested together with the lse values); a row whose unit
 // was not split (its piece wrote the output directly) costs one read. A fixed
 // grid of 8 blocks per SM strides over the rows. The kernel is launched with
 // programmatic stream serialization and waits for the decode grid first.
@@ -41,18 +42,36 @@ __global__ void __launch_bounds__(kCombineThreads) mla_combine_kernel(
     for (int i = 0; i < 4; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     float L = -INFINITY;  // no split at all: an empty key set (out 0, lse -inf)
     if (n >= 2) {
+      // split s of the row: lse at lse_u[s * rows], partial row at o_u[s * o_stride]
+      const float* lse_u = part_lse + (size_t)s0 * rows + r;
+      const float4* o_u = reinterpret_cast<const float4*>(part_o + ((size_t)s0 * rows + r) * kDv) + lane;
+      const size_t o_stride = (size_t)rows * (kDv / 4);
+      // the first two partial rows are requested with the lse values (most
+      // split units have two pieces), not after the weights are known
+      float4 o0[4], o1[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        o0[i] = o_u[32 * i];
+        o1[i] = o_u[o_stride + 32 * i];
+      }
       float m = -INFINITY;
-      for (int s = 0; s < n; ++s) m = fmaxf(m, part_lse[(size_t)(s0 + s) * rows + r]);
+      for (int s = 0; s < n; ++s) m = fmaxf(m, lse_u[(size_t)s * rows]);
       if (m != -INFINITY) {
         float sum = 0.f;
-        for (int s = 0; s < n; ++s) sum += expf(part_lse[(size_t)(s0 + s) * rows + r] - m);
+        for (int s = 0; s < n; ++s) sum += expf(lse_u[(size_t)s * rows] - m);
         L = m + logf(sum);
-        for (int s = 0; s < n; ++s) {
-          const float w = expf(part_lse[(size_t)(s0 + s) * rows + r] - L);
-          const float4* src = reinterpret_cast<const float4*>(part_o + ((size_t)(s0 + s) * rows + r) * kDv);
+        // splits in order, acc += w_s o_s from zero
+        const float w0 = expf(lse_u[0] - L), w1 = expf(lse_u[rows] - L);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          acc[i].x += w0 * o0[i].x; acc[i].y += w0 * o0[i].y; acc[i].z += w0 * o0[i].z; acc[i].w += w0 * o0[i].w;
+          acc[i].x += w1 * o1[i].x; acc[i].y += w1 * o1[i].y; acc[i].z += w1 * o1[i].z; acc[i].w += w1 * o1[i].w;
+        }
+        for (int s = 2; s < n; ++s) {
+          const float w = expf(lse_u[(size_t)s * rows] - L);
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            const float4 o = src[lane + 32 * i];
+            const float4 o = o_u[s * o_stride + 32 * i];
             acc[i].x += w * o.x; acc[i].y += w * o.y; acc[i].z += w * o.z; acc[i].w += w * o.w;
           }
         }
