@@ -50,16 +50,42 @@ KERNEL_SOURCE = {"mla_decode_pair_kernel": "mla_decode_pair.cu", "mla_decode_ker
                  "mla_decode_page_kernel": "mla_decode_page.cu"}
 
 
+def strip_c_comments(src: str) -> str:
+    """C/C++ source without its comments and blank lines, trailing spaces
+    dropped; string and character literals (inline PTX) are kept as written."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        j = min((k for k in (src.find("//", i), src.find("/*", i), src.find('"', i), src.find("'", i)) if k >= 0),
+                default=n)
+        out.append(src[i:j])
+        if j >= n:
+            break
+        if src.startswith("//", j):
+            k = src.find("\n", j)
+            i = n if k < 0 else k
+        elif src.startswith("/*", j):
+            k = src.find("*/", j + 2)
+            i = n if k < 0 else k + 2
+        else:  # a literal: copy it through its closing quote
+            q, k = src[j], j + 1
+            while k < n and src[k] != q:
+                k += 2 if src[k] == "\\" else 1
+            out.append(src[j:k + 1])
+            i = k + 1
+    lines = (line.rstrip() for line in "".join(out).split("\n"))
+    return "\n".join(line for line in lines if line)
+
+
 def kernel_source_hash(kernel: str) -> str:
     """Hash of what one decode kernel is built from: its own .cu file and the
-    shared headers (the scheduler, combine and host-side files do not change
-    the kernel's memory traffic)."""
+    shared headers, without comments (the scheduler, combine and host-side
+    files, and comments, do not change the kernel's memory traffic)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "head_latent_attention_get_b200", "csrc")
     for f in sorted(os.listdir(csrc)):
         if f.endswith(".cuh") or f == KERNEL_SOURCE[kernel]:
-            with open(os.path.join(csrc, f), "rb") as fh:
-                h.update(fh.read())
+            with open(os.path.join(csrc, f), encoding="utf-8") as fh:
+                h.update(strip_c_comments(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

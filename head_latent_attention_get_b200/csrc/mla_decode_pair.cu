@@ -17,7 +17,8 @@
 //   softmax     thread (row, half) of the CTA reads its row's 128 scores of
 //               token half `half`; the row max is agreed between the two
 //               threads of a row through shared memory, once per step. The
-//               probabilities go straight to one of two P buffers.
+//               probabilities go straight to the P buffer once the
+//               previous step's O product has read it.
 //   O = P V     pair MMA M=128 x N=256 (value dims, 128 per CTA) x K=256
 //               tokens, twice (dims 0-255 and 256-511). P is this CTA's 64
 //               rows (K-major); V is read MN-major straight from the

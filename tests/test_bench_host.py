@@ -33,3 +33,15 @@ def test_roofline_fraction_of_the_kernel_time():
     assert r["bound"] == "hbm"
     assert abs(r["achieved"] - work["bytes"] / 1e-4 / 1e9) < 1e-6 * r["achieved"]
     assert abs(r["frac"] - r["achieved"] / PEAKS["hbm_gbs"]) < 1e-12
+
+
+def test_kernel_hash_ignores_comments_but_not_code():
+    code = "int f(int x) { return x + 1; }  // add one\n"
+    a = B.strip_c_comments("/* header\n   two lines */\n" + code)
+    b = B.strip_c_comments("// another header\n\n" + code.replace("// add one", "/* plus one */"))
+    assert a == b == "int f(int x) { return x + 1; }"
+    assert B.strip_c_comments(code.replace("x + 1", "x + 2")) != a
+    # comment markers inside string literals (inline PTX) are code
+    ptx = 'asm volatile("mov.b32 %0, 1; // kept /* kept */" : "=r"(v));'
+    assert B.strip_c_comments(ptx) == ptx
+    assert B.strip_c_comments("char q = '\"'; int y; // c") == "char q = '\"'; int y;"
